@@ -1,0 +1,349 @@
+"""Benchmark: one paged-attention step (cache write of the new tokens + attention)
+on the decode workload, TinyLlama-1.1B attention shape (32 q / 4 kv heads,
+head_dim 64, 64 sequences of context U[128, 2048], 16-token blocks, 100k-block
+pool), bf16, synthetic N(0,1) data.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  `value` is decode KV GB/s: the K/V bytes the
+step's attention must read (sum over sequences of seq_len * 2 * Hkv * D * 2 B,
+summed over ranks) divided by the device time of a step (max over ranks).  L2
+is flushed (a 512 MiB write) before every timed step and the flush is not
+timed.  `--impl reference` times the CPU oracle on a bounded sample of the same
+workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode paged-attn KV GB/s (% of HBM peak); mixed-step query tokens/s"
+WORKLOAD = "decode_tinyllama"
+FLUSH_BYTES = 512 << 20
+
+
+def kv_bytes(step, seqs=None) -> int:
+    """Algorithmic K+V bytes one step's attention reads: every key of every
+    sequence once per kv-head."""
+    import numpy as np
+    lens = step.seq_lens if seqs is None else step.seq_lens[seqs]
+    elem = 4 if step.dtype == "f32" else 2
+    return int(np.sum(lens.astype(np.int64))) * 2 * step.num_kv_heads * step.head_dim * elem
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 20):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", str(period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)  # let it start sampling
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (identity on one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle legs
+
+def oracle_sample(step, target_s: float, threads: int):
+    """Time the oracle on the first n sequences (all their query rows), n grown
+    until one pass takes about target_s seconds.  Returns (GB/s, n, seconds)."""
+    import numpy as np
+    import oracle
+    from tests.oracle_side import oracle_state
+    st = oracle_state(step)
+    qsl = st["query_start_loc"]
+
+    def run(n):
+        tok = np.repeat(np.arange(int(qsl[n]), dtype=np.int64), step.num_q_heads)
+        head = np.tile(np.arange(step.num_q_heads, dtype=np.int32), int(qsl[n]))
+        t0 = time.perf_counter()
+        oracle.paged_attention_rows(step.q, st["k_cache"], st["v_cache"], st["block_tables"],
+                                    step.seq_lens, qsl, tok, head,
+                                    num_q_heads=step.num_q_heads, scale=step.scale,
+                                    num_threads=threads)
+        return time.perf_counter() - t0
+
+    n = 1
+    dt = run(n)
+    while dt < target_s and n < step.num_seqs:
+        n = min(step.num_seqs, max(n + 1, int(n * target_s / max(dt, 1e-3))))
+        dt = run(n)
+    # a whole step shorter than the target: repeat it until the target is reached
+    passes, total = 1, dt
+    while total < target_s:
+        total += run(n)
+        passes += 1
+    return kv_bytes(step, np.arange(n)) * passes / total / 1e9, n, total, run, passes
+
+
+def bench_reference(args) -> None:
+    """The CPU oracle as the reference arm: each step is one pass over a bounded
+    sample of the workload, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from paged_kv_cache_469_b200.inputs import workload
+    step = workload(WORKLOAD)
+    threads = os.cpu_count() or 1
+    gbs, n, dt, run, _ = oracle_sample(step, target_s=1.0, threads=threads)
+    import numpy as np
+    for _ in range(args.warmup):
+        run(n)
+    times = [run(n) for _ in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = kv_bytes(step, np.arange(n)) / (ms / 1e3) / 1e9
+    sample = (f"first {n} of {step.num_seqs} sequences, all {step.num_q_heads} q-heads, "
+              f"fp64 oracle, {threads} threads")
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "num_seqs": step.num_seqs,
+                       "context": "U[128,2048]", "num_q_heads": 32, "num_kv_heads": 4,
+                       "head_dim": 64, "block_size": 16, "num_blocks": step.num_blocks},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def bench_ours(args) -> None:
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_469_b200 import lib
+    from paged_kv_cache_469_b200.inputs import workload
+    from paged_kv_cache_469_b200.step import DeviceStep
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    lib.library()
+    step = workload(WORKLOAD)
+    ds = DeviceStep(step, device=str(dev))
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    # ---- device-resident step: warm-up, then K timed steps (L2 flushed before each)
+    for _ in range(args.warmup):
+        ds.run()
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local) if rank == 0 or world > 1 else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        ds.write_new_tokens()
+        ev[i][1].record(stream)
+        ds.attention()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / args.steps
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    step_ms_max = max_over_ranks(step_ms, world)
+    attn_ms_max = max_over_ranks(attn_ms, world)
+    bytes_rank = kv_bytes(step)
+    bytes_all = sum_over_ranks(bytes_rank, world)
+    value = bytes_all / (step_ms_max / 1e3) / 1e9
+
+    # ---- end to end through the public API from pinned host buffers
+    host_in = {k: torch.from_numpy(np.ascontiguousarray(a)) for k, a in (
+        ("q", step.q), ("k_new", step.k_new), ("v_new", step.v_new),
+        ("slot_mapping", ds.plan.slot_mapping), ("block_tables", ds.plan.block_tables),
+        ("seq_lens", ds.plan.seq_lens), ("query_start_loc", ds.plan.query_start_loc))}
+    host_in = {k: v.pin_memory() for k, v in host_in.items()}
+    host_out = torch.empty(ds.out.shape, dtype=torch.int16).pin_memory()
+    dev_view = {"q": ds.q.view(torch.int16), "k_new": ds.k_new.view(torch.int16),
+                "v_new": ds.v_new.view(torch.int16), "slot_mapping": ds.slot_mapping,
+                "block_tables": ds.block_tables, "seq_lens": ds.seq_lens,
+                "query_start_loc": ds.query_start_loc}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k, hv in host_in.items():
+            dev_view[k].copy_(hv.view(dev_view[k].dtype), non_blocking=True)
+        ds.run()
+        host_out.copy_(ds.out.view(torch.int16), non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        ev2[i][0].record(stream)
+        e2e_step()
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / args.steps, world)
+    e2e_value = bytes_all / (e2e_ms / 1e3) / 1e9
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    peaks = load_peaks()
+    achieved = bytes_rank / (attn_ms_max / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "kernel": "decode_splitk_kernel<64,false>",
+                "peak_source": f"{peaks['source']} HBM copy bandwidth (burst)",
+                "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        gbs, n, dt, _, passes = oracle_sample(step, target_s=10.0, threads=threads)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {n} of {step.num_seqs} sequences (all q-heads), {passes} "
+                         f"passes, {dt:.1f} s"}
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "num_seqs": step.num_seqs,
+                       "context": "U[128,2048]", "num_q_heads": 32, "num_kv_heads": 4,
+                       "head_dim": 64, "block_size": 16, "num_blocks": step.num_blocks,
+                       "kv_bytes_per_step_per_gpu": bytes_rank,
+                       "l2": "flushed (512 MiB write) before every timed step",
+                       "parallelism": f"{world} independent replicas"},
+            "attention_ms": round(attn_ms_max, 5),
+            "gpu_launches": 2 * args.steps,
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "roofline": roofline, "cpu_baseline": cpu, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * pa.h -- C ABI of the B200 (sm_100a) paged-attention library libpa.so.
+ *
+ * The method (page "LLM推論エンジンvLLMの内部構造を徹底解説", techfeed.io summary of
+ * "Inside vLLM: Anatomy of a High-Throughput LLM Inference System"):
+ *   section "PagedAttentionの仕組み" -- the KV cache is a pool of fixed-size
+ *   blocks (16 tokens by default), each request owning a list of blocks (its
+ *   row of the block table); a step's sequences are flattened into one
+ *   super-sequence, and position indices plus a mask let each sequence attend
+ *   only to its own tokens.
+ *   section "高度な機能群" -- chunked prefill (a chunk attends to the context
+ *   cached before it) and prefix caching (several block lists point at the
+ *   same physical blocks).
+ *   section "エンジンの中核" -- prefill is compute-bound, decode (the newest
+ *   token only, against the cache) is memory-bandwidth-bound, and one step may
+ *   mix both.
+ *
+ * Conventions of every call:
+ *   - Every tensor pointer is DEVICE memory owned by the caller, contiguous,
+ *     row-major, 16-byte aligned.  The library allocates nothing and keeps no
+ *     state between calls; the caller's workspace holds all scratch.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Argument checks run on the host before any
+ *     launch and return PA_ERR_INVALID / PA_ERR_UNSUPPORTED with nothing
+ *     launched; PA_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *   - Nothing traps on the device.  Slots or block ids outside the pool are
+ *     never dereferenced (see each call).
+ *   - dtype is the element type of q, k, v, the caches and out alike.
+ *
+ * Cache layout (the pages give none; this library's reading):
+ *   k_cache, v_cache: [num_blocks][num_kv_heads][block_size][head_dim]; the
+ *   16 tokens of one (block, kv-head) are one contiguous 2 KiB (D=64) or 4 KiB
+ *   (D=128) bf16 tile.  Slot s is block s / block_size, offset s % block_size.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* = cudaStream_t without pulling in the CUDA headers */
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = -1,     /* a size, pointer or alignment is wrong */
+  PA_ERR_UNSUPPORTED = -2, /* valid, but not a shape this library implements */
+  PA_ERR_CUDA = -3         /* a kernel launch failed */
+} pa_status;
+
+typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+
+/* Human-readable name of a pa_status value (static string). */
+const char* pa_status_string(int status);
+
+/*
+ * pa_reshape_and_cache -- write this step's new K/V rows into their cache slots.
+ *
+ * For every i < num_tokens with slot = slot_mapping[i] in [0, num_blocks *
+ * block_size):  k_cache[slot / block_size][h][slot % block_size][:] = k[i][h][:]
+ * and the same for v, for every kv-head h.  A slot outside that range (e.g. a
+ * negative padding slot) skips the row.  The copy is bit-exact.  Two tokens
+ * naming the same slot race (caller error).
+ *
+ *   k, v          [num_tokens][num_kv_heads][head_dim]
+ *   k_cache,
+ *   v_cache       [num_blocks][num_kv_heads][block_size][head_dim] (written)
+ *   slot_mapping  int64 [num_tokens]
+ * Supported: head_dim in {64, 128}; block_size 16; dtype f32 or bf16.
+ * Slot of position p of a request: block_table[p / 16] * 16 + p % 16
+ * (section "PagedAttentionの仕組み": blocks of 16 tokens, filled in order).
+ */
+int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                         const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                         struct CUstream_st* stream);
+
+/*
+ * Bytes of workspace pa_attention_varlen needs for a step of at most
+ * num_seqs sequences, no sequence longer than max_seq_len tokens: fp32
+ * split-K partials (running max, sum and unnormalised output per partition
+ * of a sequence's keys) plus one int32 arrival counter per (sequence,
+ * kv-head).  Always at least 256 for valid arguments; 0 means invalid
+ * arguments.
+ */
+size_t pa_attention_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int max_seq_len);
+
+/*
+ * Zero a workspace before its first use (a cudaMemsetAsync on `stream`).
+ * Every pa_attention_varlen call leaves the counters at zero again, so this is
+ * needed once per workspace allocation.
+ */
+int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_st* stream);
+
+/*
+ * pa_attention_varlen -- paged attention over one flattened step.
+ *
+ * Sequence s owns query rows query_start_loc[s] .. query_start_loc[s+1]-1 of q
+ * (q_len = their count) and seq_lens[s] keys (all of its tokens, this step's
+ * new ones included; their K/V must already be in the cache, written by
+ * pa_reshape_and_cache).  Query j of sequence s sits at position
+ * seq_lens[s] - q_len + j and attends to keys 0..that position of its own
+ * sequence, read through block_tables[s] (a decode is q_len = 1; a prefill
+ * chunk over cached context is q_len > 1 with seq_lens[s] > q_len).  q-head h
+ * reads kv-head h / (num_q_heads / num_kv_heads).
+ *
+ *   out[t][h][:] = sum_k softmax_k(scale * q[t][h] . K_k) V_k
+ *
+ *   out            [num_tokens][num_q_heads][head_dim] (written)
+ *   q              [num_tokens][num_q_heads][head_dim]
+ *   k_cache,
+ *   v_cache        [num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_tables   int32 [num_seqs][max_blocks_per_seq]; entries beyond
+ *                  ceil(seq_lens[s] / block_size) are never read; an entry
+ *                  outside [0, num_blocks) is never dereferenced (its keys
+ *                  are left out of the softmax: the result is then not
+ *                  meaningful, but no memory outside the pool is touched)
+ *   seq_lens       int32 [num_seqs]
+ *   query_start_loc int32 [num_seqs + 1], query_start_loc[0] = 0,
+ *                  nondecreasing, query_start_loc[num_seqs] = num_tokens
+ *   max_query_len, max_seq_len  host-side upper bounds over the step (they
+ *                  size the launch grids; a sequence beyond them is caller
+ *                  error and may be left unwritten)
+ *   workspace      at least pa_attention_workspace_size(num_seqs, num_q_heads,
+ *                  num_kv_heads, head_dim, max_seq_len) bytes, zeroed once by
+ *                  pa_workspace_init; one workspace serves one call at a time
+ *   seq_lens_host, query_start_loc_host  optional (NULL) host copies of the
+ *                  two device arrays: when given, the call checks them and
+ *                  launches only the kernels the step needs
+ *
+ * Decode-class sequences (q_len * num_q_heads / num_kv_heads <= 16 query
+ * rows per kv-head) run the split-K bandwidth-bound kernel; longer prefill
+ * chunks run the tensor-core kernel.  fp32 steps run a CUDA-core kernel.
+ * Supported: head_dim in {64, 128}; block_size 16; num_q_heads a multiple of
+ * num_kv_heads with at most 16 q-heads per kv-head; dtype f32 or bf16.
+ */
+int pa_attention_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, int max_blocks_per_seq,
+                        const int32_t* seq_lens, const int32_t* query_start_loc, int num_seqs,
+                        int num_tokens, int max_query_len, int max_seq_len, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                        const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
+                        struct CUstream_st* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

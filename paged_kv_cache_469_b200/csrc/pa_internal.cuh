@@ -1,0 +1,64 @@
+// pa_internal.cuh -- launch parameters and launchers shared by the kernels of
+// libpa.so and its C-ABI front end (pa_api.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pa {
+
+constexpr int kBlockSize = 16;       // tokens per cache block (the pages' default)
+constexpr int kDecodeRows = 16;      // query rows per kv-head one decode CTA holds (MMA M)
+constexpr int kDecodeWarps = 4;      // warps of a decode CTA
+
+// Everything one attention launch reads; the same struct serves every kernel.
+struct AttnParams {
+  void* out;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  const int32_t* query_start_loc;
+  int max_blocks_per_seq;
+  int num_seqs;
+  int num_tokens;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;  // num_q_heads / num_kv_heads
+  int num_blocks;
+  float scale;       // softmax scale (natural-log base)
+  float scale_log2;  // scale * log2(e), for exp2-based softmax
+  // split-K decode
+  int part_tokens;   // keys per partition (multiple of 16)
+  int max_parts;     // partitions the workspace holds per (sequence, kv-head)
+  float* ws_o;       // [num_seqs*Hkv][max_parts][16][D] unnormalised partial outputs
+  float* ws_ml;      // [num_seqs*Hkv][max_parts][16][2] running max (log2 units), sum
+  int* ws_counter;   // [num_seqs*Hkv] arrival counters, zero between calls
+};
+
+// Workspace layout shared by the size query and the launch.
+struct WorkspaceLayout {
+  int part_tokens;
+  int max_parts;
+  size_t counter_off, o_off, ml_off, total;
+};
+WorkspaceLayout workspace_layout(int num_seqs, int num_kv_heads, int head_dim, int max_seq_len);
+
+// Launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                                     const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int head_dim, int num_blocks,
+                                     int elem_bytes, cudaStream_t stream);
+
+// CUDA-core kernel: every query row whose sequence has more than
+// min_rows_per_kv_head query rows per kv-head (0 = all rows).
+cudaError_t launch_attention_simple(const AttnParams& p, int head_dim, bool is_bf16,
+                                    int min_rows_per_kv_head, cudaStream_t stream);
+
+// Split-K decode kernel (bf16): sequences with q_len * group <= 16.
+cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
+                                 cudaStream_t stream);
+
+}  // namespace pa

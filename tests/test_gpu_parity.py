@@ -1,0 +1,242 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+Bars: the cache write is bit-exact over the whole pool; fp32 outputs within
+1e-4 absolute; bf16 outputs within 2e-2 + 1e-2 * |ref| elementwise, ref being
+the oracle's fp64 value before any rounding.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_469_b200.inputs import make_step, random_step, workload
+from tests.oracle_side import oracle_outputs, oracle_state
+
+pytestmark = pytest.mark.gpu
+
+NTHREADS = max(1, os.cpu_count() or 1)
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    if dtype == "f32":
+        assert err.max(initial=0.0) <= 1e-4, f"{what}: max abs err {err.max()}"
+    else:
+        bound = 2e-2 + 1e-2 * np.abs(ref)
+        bad = err > bound
+        assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} elements out of tolerance, "
+                               f"worst {err.max()}")
+
+
+def run_and_check(step, *, full=True, rows=None, check_cache=True, host_hints=True):
+    from paged_kv_cache_469_b200.step import DeviceStep
+    ds = DeviceStep(step)
+    ds.run(host_hints=host_hints)
+    torch.cuda.synchronize()
+    st = oracle_state(step)
+    if check_cache:
+        assert _bits(ds.k_cache).tobytes() == st["k_cache"].tobytes(), "k_cache differs"
+        assert _bits(ds.v_cache).tobytes() == st["v_cache"].tobytes(), "v_cache differs"
+    got = ds.out_f64()
+    if full:
+        ref = oracle_outputs(step, st, num_threads=NTHREADS)
+        assert_close(got, ref, step.dtype, step.name)
+    if rows is not None:
+        tok, head = rows
+        ref = oracle.paged_attention_rows(step.q, st["k_cache"], st["v_cache"],
+                                          st["block_tables"], step.seq_lens,
+                                          st["query_start_loc"], tok, head,
+                                          num_q_heads=step.num_q_heads, scale=step.scale,
+                                          num_threads=NTHREADS)
+        assert_close(got[tok, head], ref, step.dtype, step.name + " (sampled rows)")
+    # split-K counters are back at zero for the next call
+    n = step.num_seqs * step.num_kv_heads * 4
+    assert int(ds.workspace[:n].count_nonzero()) == 0
+    return ds, st
+
+
+def test_tiny_fp32_workload():
+    run_and_check(workload("tiny_f32"))
+
+
+def test_tiny_fp32_without_host_hints():
+    run_and_check(workload("tiny_f32"), host_hints=False)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("heads", [(8, 1), (8, 2), (4, 4), (32, 4), (16, 1)])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_random_mixed_steps_bf16(d, heads, seed):
+    hq, hkv = heads
+    step = random_step(100 + seed, dtype="bf16", num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+                       num_seqs=6, max_ctx=300, max_q=40)
+    run_and_check(step)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_random_mixed_steps_fp32(d):
+    step = random_step(7, dtype="f32", num_q_heads=8, num_kv_heads=2, head_dim=d, num_seqs=5,
+                       max_ctx=200, max_q=30)
+    run_and_check(step)
+
+
+@pytest.mark.parametrize("hq,hkv,ql", [(32, 4, 2), (32, 8, 4), (16, 4, 3), (8, 8, 16),
+                                       (16, 16, 1), (16, 1, 1)])
+def test_multi_token_decode_rows(hq, hkv, ql):
+    """Decode-class sequences whose q_len * group fills 9..16 MMA rows (speculative
+    verification shapes), mixed with plain decodes."""
+    lens = [1000, 37, 300, 16, 17]
+    qls = [ql, 1, ql, 1, ql]
+    step = make_step(name="mtd", dtype="bf16", num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+                     num_blocks=200, seq_lens=lens, query_lens=qls, seed=5)
+    run_and_check(step)
+
+
+def test_long_split_k_and_edge_lengths():
+    """Many partitions (L up to 5000), one-key sequences, ragged last blocks,
+    empty sequences (q_len 0) between non-empty ones."""
+    lens = [5000, 1, 2, 15, 16, 17, 0, 4097, 33, 3]
+    qls = [1, 1, 2, 1, 16, 17, 0, 1, 0, 3]
+    step = make_step(name="edges", dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=64,
+                     num_blocks=800, seq_lens=lens, query_lens=qls, seed=8)
+    run_and_check(step)
+    run_and_check(step, host_hints=False)
+
+
+def test_pool_edge_blocks():
+    """The first and last block of the pool are handed out."""
+    step = make_step(name="pooledge", dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=128,
+                     num_blocks=10, seq_lens=[40, 100], query_lens=[1, 30], seed=3)
+    step.free_queue = np.array([9, 0, 5, 1, 8, 2, 7, 3, 6, 4], dtype=np.int32)
+    run_and_check(step)
+
+
+def test_decode_tinyllama_full():
+    run_and_check(workload("decode_tinyllama"))
+
+
+def _sample_rows(step, rng, per_seq_tokens=2, heads=4):
+    qsl = oracle.query_start_loc(step.query_lens)
+    toks, hs = [], []
+    for s in range(step.num_seqs):
+        ql = int(step.query_lens[s])
+        if ql == 0:
+            continue
+        picks = {0, ql - 1} | set(rng.integers(0, ql, size=per_seq_tokens).tolist())
+        for j in sorted(picks):
+            for h in rng.choice(step.num_q_heads, size=heads, replace=False):
+                toks.append(int(qsl[s]) + j)
+                hs.append(int(h))
+    return np.array(toks, np.int64), np.array(hs, np.int32)
+
+
+@pytest.mark.parametrize("name", ["mixed_llama3_8b", "prefix_decode_llama3_8b",
+                                  "long_decode_llama3_8b"])
+def test_full_size_workloads_sampled(name):
+    step = workload(name)
+    rows = _sample_rows(step, np.random.default_rng(1), heads=2 if name != "long_decode_llama3_8b"
+                        else 8)
+    run_and_check(step, full=False, rows=rows, check_cache=(name != "long_decode_llama3_8b"))
+
+
+# ---------------------------------------------------------------- invariances on the GPU
+
+def _gpu_out(step, host_hints=True):
+    from paged_kv_cache_469_b200.step import DeviceStep
+    ds = DeviceStep(step)
+    ds.run(host_hints=host_hints)
+    torch.cuda.synchronize()
+    return _bits(ds.out)
+
+
+def test_block_permutation_bit_identical():
+    step = random_step(61, dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                       num_seqs=6, max_ctx=600, max_q=40)
+    base = _gpu_out(step)
+    step.free_queue = np.random.default_rng(9).permutation(step.num_blocks).astype(np.int32)
+    assert _gpu_out(step).tobytes() == base.tobytes()
+
+
+def test_shared_prefix_equals_private_copies_gpu():
+    st = random_step(71, dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                     num_seqs=5, max_ctx=200, max_q=1, shared_prefix_tokens=256)
+    shared = _gpu_out(st)
+    priv = make_step(name="priv", dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                     num_blocks=st.num_blocks + 5 * 16, seq_lens=st.seq_lens,
+                     query_lens=st.query_lens, seed=st.seed)
+    c_off = np.concatenate([[0], np.cumsum(st.ctx_count)])
+    ks, vs = [], []
+    for s in range(st.num_seqs):
+        if s > 0:
+            ks.append(st.k_ctx[:256])
+            vs.append(st.v_ctx[:256])
+        ks.append(st.k_ctx[c_off[s]:c_off[s + 1]])
+        vs.append(st.v_ctx[c_off[s]:c_off[s + 1]])
+    priv.k_ctx, priv.v_ctx = np.concatenate(ks), np.concatenate(vs)
+    priv.q, priv.k_new, priv.v_new = st.q, st.k_new, st.v_new
+    assert _gpu_out(priv).tobytes() == shared.tobytes()
+
+
+def test_sequence_order_does_not_change_rows():
+    step = random_step(81, dtype="bf16", num_q_heads=16, num_kv_heads=4, head_dim=64,
+                       num_seqs=5, max_ctx=400, max_q=24)
+    base = _gpu_out(step)
+    perm = np.array([3, 1, 4, 0, 2])
+    q_off = np.concatenate([[0], np.cumsum(step.query_lens)])
+    c_off = np.concatenate([[0], np.cumsum(step.ctx_count)])
+    re = make_step(name="re", dtype="bf16", num_q_heads=16, num_kv_heads=4, head_dim=64,
+                   num_blocks=step.num_blocks, seq_lens=step.seq_lens[perm],
+                   query_lens=step.query_lens[perm], seed=1)
+    take = lambda a, off: np.concatenate([a[off[s]:off[s + 1]] for s in perm])
+    re.q, re.k_new, re.v_new = take(step.q, q_off), take(step.k_new, q_off), take(step.v_new, q_off)
+    re.k_ctx, re.v_ctx = take(step.k_ctx, c_off), take(step.v_ctx, c_off)
+    out = _gpu_out(re)
+    r_off = np.concatenate([[0], np.cumsum(re.query_lens)])
+    for i, s in enumerate(perm):
+        assert out[r_off[i]:r_off[i + 1]].tobytes() == base[q_off[s]:q_off[s + 1]].tobytes()
+
+
+def test_chunked_prefill_matches_one_shot_gpu():
+    """Prefill 700 tokens at once vs 3 chunks with cache writes in between."""
+    from paged_kv_cache_469_b200.inputs import bf16_bits_to_f32
+    one = make_step(name="one", dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                    num_blocks=64, seq_lens=[700], query_lens=[700], seed=12)
+    full = _gpu_out(one)
+    kall, vall = one.k_new, one.v_new
+    start = 0
+    for n in (256, 300, 144):
+        ch = make_step(name="chunk", dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                       num_blocks=64, seq_lens=[start + n], query_lens=[n], seed=12)
+        ch.free_queue = one.free_queue
+        ch.q = one.q[start:start + n]
+        ch.k_ctx, ch.v_ctx = kall[:start], vall[:start]
+        ch.k_new, ch.v_new = kall[start:start + n], vall[start:start + n]
+        got = bf16_bits_to_f32(_gpu_out(ch)).astype(np.float64)
+        ref = bf16_bits_to_f32(full[start:start + n]).astype(np.float64)
+        np.testing.assert_allclose(got, ref, atol=2e-2, rtol=1e-2)
+        start += n
+
+
+def test_zero_token_call_is_a_no_op():
+    from paged_kv_cache_469_b200 import lib
+    dev = "cuda"
+    kc = torch.zeros(4, 2, 16, 64, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(0, 8, 64, dtype=torch.bfloat16, device=dev)
+    lib.attention_varlen(out, out, kc, kc, torch.zeros(1, 1, dtype=torch.int32, device=dev),
+                         torch.zeros(1, dtype=torch.int32, device=dev),
+                         torch.zeros(2, dtype=torch.int32, device=dev), max_query_len=0,
+                         max_seq_len=0, scale=0.125, workspace=None)
+    lib.reshape_and_cache(out[:, :2], out[:, :2], kc, kc,
+                          torch.zeros(0, dtype=torch.int64, device=dev))
+    torch.cuda.synchronize()
