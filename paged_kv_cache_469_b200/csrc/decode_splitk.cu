@@ -11,22 +11,30 @@
 // byte is read from HBM once per kv-head.  Warp w of the CTA takes blocks
 // w, w+4, ... of the partition.
 //
-// Per 16-token block (one (block, kv-head) tile: 16 x D bf16, contiguous):
-//   S[16 rows x 16 keys]  = Q . K^T    two mma.m16n8k16 per 16 dims of D
+// Staging.  Each warp streams its blocks through a private ring of kStages
+// shared-memory slots (one (block, kv-head) K tile + V tile per slot) with
+// 16-byte cp.async copies, kStages-1 blocks in flight ahead of the math.  The
+// 16-byte chunks of every tile row are XOR-swizzled on the way in so that the
+// fragment reads below hit 32 distinct banks.
+//
+// Per 16-token block:
+//   S[16 rows x 16 keys]  = Q . K^T    mma.m16n8k16, two per 16 dims of D
 //   online softmax (running max / sum in fp32, exp2 with log2(e) folded in)
 //   O[16 rows x D]       += P . V      D/8 mma.m16n8k16
-// Operands come straight from HBM into registers with 16-byte loads, no shared
-// memory: the dot product's D axis is permuted identically on Q and K so that
-// every lane's B-operand words are 8 consecutive bf16 of one key row, and the
+// The dot product's D axis is permuted identically on Q and K so that every
+// lane's B-operand words are 8 consecutive bf16 of one key row, and the
 // output's D axis is permuted so that every lane's V words are 8 consecutive
-// bf16 of one key row (the permutation is undone when the output is stored).
-// The next block's K/V loads are issued before the current block's math.
+// bf16 of one key row (undone when the output is stored).
 //
 // Split-K.  A CTA reduces its 4 warps' (max, sum, O) in shared memory.  A
 // sequence that fits one partition writes its output directly; otherwise each
 // partition stores its fp32 partial in the workspace and bumps a per
 // (sequence, kv-head) counter; the CTA that arrives last merges all partials
 // and resets the counter.  No CTA ever waits for another.
+//
+// The kernel is launched as a programmatic dependent of whatever precedes it
+// on the stream (typically the cache write), so its launch overlaps that
+// kernel's tail; it reads nothing before griddepcontrol.wait.
 #include <math.h>
 
 #include "pa_internal.cuh"
@@ -47,36 +55,64 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void* ptr) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(ptr));
-  return r;
+__device__ __forceinline__ void cp_async16(uint32_t smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// Output column c (0..7) of n-tile nt sits at dimension
-//   64 * (nt / 8) + 8 * c + nt % 8
-// so a lane that owns columns 2*q4, 2*q4+1 of every n-tile owns, per 64-wide
-// half of D, the 16 consecutive dimensions 16*q4 .. 16*q4+15.
-template <int D>
-__device__ __forceinline__ int out_dim(int nt, int c) {
-  return 64 * (nt / 8) + 8 * c + (nt % 8);
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
 }
 
-template <int D, bool kRows16>
+// XOR applied to the 16-byte chunk index of tile row `row` (K and V tiles).
+// K rows are read two at a time (rows 2k, 2k+1, chunk 4j..4j+3): flip the
+// half of the 128-byte line on odd rows.  V rows are read four at a time
+// (rows of equal parity), one chunk each: spread them by row bits 1-2.
+__device__ __forceinline__ int k_swz(int row) { return (row & 1) << 2; }
+__device__ __forceinline__ int v_swz(int row) { return row & 6; }
+
+// Output column c (0..7) of n-tile nt sits at dimension 64*(nt/8) + 8*c + nt%8,
+// so a lane owning columns 2*q4, 2*q4+1 of every n-tile owns, per 64-wide
+// half of D, the 16 consecutive dimensions 16*q4 .. 16*q4+15.
+__device__ __forceinline__ int out_dim(int nt, int c) { return 64 * (nt / 8) + 8 * c + (nt % 8); }
+
+template <int D>
+struct DecodeSmem {
+  static constexpr int kChunks = D / 8;                 // 16-byte chunks per tile row
+  static constexpr int kTileBytes = kBlockSize * D * 2;  // one (block, kv-head) tile
+  static constexpr int kSlotBytes = 2 * kTileBytes;      // K tile + V tile
+};
+
+template <int D, bool kRows16, int kStages>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
 decode_splitk_kernel(const AttnParams p) {
-  constexpr int NJ = D / 32;  // 16-byte K words per key row per lane
-  constexpr int NV = D / 64;  // 16-byte V words per key row per lane
+  constexpr int NJ = D / 32;  // 16-byte K chunks per key row a lane reads
+  constexpr int NV = D / 64;  // 16-byte V chunks per key row a lane reads
   constexpr int NT = D / 8;   // n-tiles of the P.V product
   constexpr int NC = D / 16;  // k-chunks of the Q.K^T product
+  using SM = DecodeSmem<D>;
+  constexpr int kChunks = SM::kChunks;
+  constexpr int kCopies = kBlockSize * kChunks / 32;  // 16-byte copies per lane per tile
 
-  __shared__ float sh_o[kDecodeWarps][kDecodeRows][D];
+  extern __shared__ __align__(128) unsigned char smem[];
   __shared__ float sh_m[kDecodeWarps][kDecodeRows];
   __shared__ float sh_l[kDecodeWarps][kDecodeRows];
   __shared__ int sh_last;
@@ -84,6 +120,11 @@ decode_splitk_kernel(const AttnParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = lane >> 2, q4 = lane & 3;
   const int s = blockIdx.z, kvh = blockIdx.y, part = blockIdx.x;
+
+  // Launched as a programmatic dependent: the CTA may be resident before the
+  // preceding kernel on the stream (typically the cache write) has finished;
+  // nothing that kernel may write is read before this wait.
+  grid_dependency_wait();
 
   const int q0 = p.query_start_loc[s];
   const int ql = p.query_start_loc[s + 1] - q0;
@@ -103,19 +144,20 @@ decode_splitk_kernel(const AttnParams p) {
   const int blk_begin = t_begin / kBlockSize;
   const int blk_end = (t_end + kBlockSize - 1) / kBlockSize;
 
-  const __nv_bfloat16* qg = (const __nv_bfloat16*)p.q;
-  const char* kc = (const char*)p.k_cache;
-  const char* vc = (const char*)p.v_cache;
-  const int64_t tile_bytes = (int64_t)kBlockSize * D * 2;          // one (block, head) tile
-  const int64_t blk_bytes = tile_bytes * p.num_kv_heads;            // one block, all heads
-  const int64_t head_off = tile_bytes * kvh;
+  // ---- this warp's block ids, one per lane (lane i <-> i-th block of the warp)
+  const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
+  const int my_nblk = (blk_end - blk_begin - warp + kDecodeWarps - 1) / kDecodeWarps;
+  int my_id = 0;
+  if (lane < my_nblk) my_id = table[blk_begin + warp + kDecodeWarps * lane];
 
-  // ---- Q as the A operand (rows r and r+8), D axis permuted as the K words
+  // ---- Q as the A operand (rows r and r+8), D axis permuted as the K chunks
+  const __nv_bfloat16* qg = (const __nv_bfloat16*)p.q;
   uint32_t qa[NC][2], qb[NC][2];
   {
     const bool va = r < rows, vb = kRows16 && (r + 8) < rows;
     const int64_t ra = va ? ((int64_t)(q0 + r / G) * p.num_q_heads + kvh * G + r % G) * D : 0;
-    const int64_t rb = vb ? ((int64_t)(q0 + (r + 8) / G) * p.num_q_heads + kvh * G + (r + 8) % G) * D : 0;
+    const int64_t rb =
+        vb ? ((int64_t)(q0 + (r + 8) / G) * p.num_q_heads + kvh * G + (r + 8) % G) * D : 0;
 #pragma unroll
     for (int jp = 0; jp < NJ; ++jp) {
       uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
@@ -130,58 +172,76 @@ decode_splitk_kernel(const AttnParams p) {
   const int lim_b = L - ql + min(r + 8, rows - 1) / G;
   const int first_masked = L - ql + 1;  // keys at or beyond this may be masked for some row
 
-  // ---- this warp's block ids, one per lane (lane i <-> i-th block of the warp)
-  const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-  const int my_nblk = (blk_end - blk_begin - warp + kDecodeWarps - 1) / kDecodeWarps;
-  int my_id = 0;
-  if (lane < my_nblk) my_id = table[blk_begin + warp + kDecodeWarps * lane];
+  const char* kc = (const char*)p.k_cache;
+  const char* vc = (const char*)p.v_cache;
+  const int64_t blk_bytes = (int64_t)SM::kTileBytes * p.num_kv_heads;
+  const int64_t head_off = (int64_t)SM::kTileBytes * kvh;
+  const uint32_t ring = (uint32_t)__cvta_generic_to_shared(smem) +
+                        warp * kStages * SM::kSlotBytes;
+
+  auto issue = [&](int i) {  // copy the warp's i-th block into slot i % kStages
+    int id = __shfl_sync(0xffffffffu, my_id, i);
+    if (id < 0 || id >= p.num_blocks) id = 0;  // never dereference outside the pool
+    const char* kt = kc + id * blk_bytes + head_off;
+    const char* vt = vc + id * blk_bytes + head_off;
+    const uint32_t ks = ring + (i % kStages) * SM::kSlotBytes;
+    const uint32_t vs = ks + SM::kTileBytes;
+#pragma unroll
+    for (int j = 0; j < kCopies; ++j) {
+      const int idx = lane + 32 * j;
+      const int row = idx / kChunks, c = idx % kChunks;
+      cp_async16(ks + (row * kChunks + (c ^ k_swz(row))) * 16, kt + idx * 16);
+      cp_async16(vs + (row * kChunks + (c ^ v_swz(row))) * 16, vt + idx * 16);
+    }
+  };
 
   float o[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
   float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
 
-  uint4 kw[2][NJ], vw[4][NV];
-  auto load_block = [&](int i, uint4 (&kd)[2][NJ], uint4 (&vd)[4][NV]) {
-    int id = __shfl_sync(0xffffffffu, my_id, i);
-    if (id < 0 || id >= p.num_blocks) id = 0;  // never dereference outside the pool
-    const char* kt = kc + id * blk_bytes + head_off;
-    const char* vt = vc + id * blk_bytes + head_off;
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int jp = 0; jp < NJ; ++jp)
-        kd[h][jp] = ldg_stream(kt + ((8 * h + r) * D + 32 * jp + 8 * q4) * 2);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = 2 * q4 + (e & 1) + 8 * (e >> 1);
-#pragma unroll
-      for (int u = 0; u < NV; ++u) vd[e][u] = ldg_stream(vt + (tok * D + 64 * u + 8 * r) * 2);
-    }
-  };
+  for (int st = 0; st < kStages - 1; ++st) {
+    if (st < my_nblk) issue(st);
+    cp_async_commit();
+  }
 
-  if (my_nblk > 0) load_block(0, kw, vw);
   for (int i = 0; i < my_nblk; ++i) {
-    uint4 kn[2][NJ], vn[4][NV];
-    const bool has_next = i + 1 < my_nblk;
-    if (has_next) load_block(i + 1, kn, vn);
+    __syncwarp();  // every lane is done reading the slot the next copy overwrites
+    if (i + kStages - 1 < my_nblk) issue(i + kStages - 1);
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();  // this lane's copies of block i have landed
+    __syncwarp();                  // ... and every other lane's
+
     const int blk = blk_begin + warp + kDecodeWarps * i;
     const int id_raw = __shfl_sync(0xffffffffu, my_id, i);
     const bool blk_ok = id_raw >= 0 && id_raw < p.num_blocks;
+    const uint32_t ks = ring + (i % kStages) * SM::kSlotBytes;
+    const uint32_t vs = ks + SM::kTileBytes;
 
     // ---- S = Q K^T (two 8-key halves of the block)
     float sc[2][4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       sc[h][0] = sc[h][1] = sc[h][2] = sc[h][3] = 0.f;
+      const int row = 8 * h + r;
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        const uint4& kx = kw[h][c / 2];
-        const uint32_t b0 = (c & 1) ? kx.z : kx.x;
-        const uint32_t b1 = (c & 1) ? kx.w : kx.y;
-        mma_16816(sc[h], qa[c][0], kRows16 ? qb[c][0] : 0u, qa[c][1], kRows16 ? qb[c][1] : 0u,
-                  b0, b1);
+      for (int jp = 0; jp < NJ; ++jp) {
+        const uint4 kx = lds128(ks + (row * kChunks + ((4 * jp + q4) ^ k_swz(row))) * 16);
+        mma_16816(sc[h], qa[2 * jp][0], kRows16 ? qb[2 * jp][0] : 0u, qa[2 * jp][1],
+                  kRows16 ? qb[2 * jp][1] : 0u, kx.x, kx.y);
+        mma_16816(sc[h], qa[2 * jp + 1][0], kRows16 ? qb[2 * jp + 1][0] : 0u,
+                  qa[2 * jp + 1][1], kRows16 ? qb[2 * jp + 1][1] : 0u, kx.z, kx.w);
       }
+    }
+    // ---- V words: keys 2q4, 2q4+1, 2q4+8, 2q4+9; 8 dims 64u+8r.. each
+    uint4 vw[4][NV];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = 2 * q4 + (e & 1) + 8 * (e >> 1);
+#pragma unroll
+      for (int u = 0; u < NV; ++u)
+        vw[e][u] = lds128(vs + (tok * kChunks + ((8 * u + r) ^ v_swz(tok))) * 16);
     }
     // ---- scale, mask, online softmax
     const int key0 = blk * kBlockSize + 2 * q4;  // keys key0, +1 (half 0), key0+8, +9 (half 1)
@@ -239,17 +299,8 @@ decode_splitk_kernel(const AttnParams p) {
       const uint32_t b1 = __byte_perm(word(vw[2][u], idx >> 1), word(vw[3][u], idx >> 1), sel);
       mma_16816(o[nt], pa0, pb1, pa2, pb3, b0, b1);
     }
-    if (has_next) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int jp = 0; jp < NJ; ++jp) kw[h][jp] = kn[h][jp];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-#pragma unroll
-        for (int u = 0; u < NV; ++u) vw[e][u] = vn[e][u];
-    }
   }
+  cp_async_wait<0>();  // no copy may still target the ring when it is reused below
 
   // ---- per-warp results to shared memory (row sums reduced over the quad)
   l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
@@ -258,6 +309,8 @@ decode_splitk_kernel(const AttnParams p) {
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
   }
+  __syncthreads();  // every warp is done with its ring
+  float(*sh_o)[kDecodeRows][D] = reinterpret_cast<float(*)[kDecodeRows][D]>(smem);
   if (q4 == 0) {
     sh_m[warp][r] = m_a; sh_l[warp][r] = l_a;
     sh_m[warp][r + 8] = m_b; sh_l[warp][r + 8] = l_b;
@@ -266,7 +319,7 @@ decode_splitk_kernel(const AttnParams p) {
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      const int d = out_dim<D>(nt, 2 * q4 + c);
+      const int d = out_dim(nt, 2 * q4 + c);
       sh_o[warp][r][d] = o[nt][c];
       if (kRows16) sh_o[warp][r + 8][d] = o[nt][2 + c];
     }
@@ -333,6 +386,27 @@ decode_splitk_kernel(const AttnParams p) {
   if (threadIdx.x == 0) p.ws_counter[unit] = 0;  // ready for the next call
 }
 
+template <int D, bool kRows16, int kStages>
+cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
+  auto kernel = decode_splitk_kernel<D, kRows16, kStages>;
+  const int ring = kDecodeWarps * kStages * DecodeSmem<D>::kSlotBytes;
+  const int merge = kDecodeWarps * kDecodeRows * D * (int)sizeof(float);
+  const int smem = ring > merge ? ring : merge;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.max_parts, p.num_kv_heads, p.num_seqs);
+  cfg.blockDim = dim3(kDecodeWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 }  // namespace
 
 cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
@@ -340,15 +414,12 @@ cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_quer
   if (p.num_seqs == 0) return cudaSuccess;
   const int max_rows = min(max_query_len * p.group, kDecodeRows);
   const bool rows16 = max_rows > 8;
-  dim3 grid(p.max_parts, p.num_kv_heads, p.num_seqs);
-  dim3 block(kDecodeWarps * 32);
-  if (head_dim == 64) {
-    if (rows16) decode_splitk_kernel<64, true><<<grid, block, 0, stream>>>(p);
-    else decode_splitk_kernel<64, false><<<grid, block, 0, stream>>>(p);
-  } else {
-    if (rows16) decode_splitk_kernel<128, true><<<grid, block, 0, stream>>>(p);
-    else decode_splitk_kernel<128, false><<<grid, block, 0, stream>>>(p);
-  }
+  cudaError_t e;
+  if (head_dim == 64)
+    e = rows16 ? launch_one<64, true, 4>(p, stream) : launch_one<64, false, 4>(p, stream);
+  else
+    e = rows16 ? launch_one<128, true, 3>(p, stream) : launch_one<128, false, 3>(p, stream);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -13,11 +13,18 @@ static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; 
 // still gives the GPU about eight waves' worth of CTAs when sequences average
 // half of max_seq_len.  (2048 = 4 warps x 32 blocks: each lane of a warp holds
 // one block id of the partition.)
+#ifndef PA_PART_MIN
+#define PA_PART_MIN 512
+#endif
+#ifndef PA_TARGET_CTAS
+#define PA_TARGET_CTAS (8 * 148)
+#endif
 static int choose_part_tokens(int num_seqs, int num_kv_heads, int max_seq_len) {
   const long units = (long)num_seqs * num_kv_heads;
-  const long target = 8L * 148;
+  const long target = PA_TARGET_CTAS;
   int part = 2048;
-  while (part > 256 && units * (((long)max_seq_len / 2 + part - 1) / part) < target) part /= 2;
+  while (part > PA_PART_MIN && units * (((long)max_seq_len / 2 + part - 1) / part) < target)
+    part /= 2;
   return part;
 }
 

@@ -16,6 +16,9 @@ reshape_and_cache_kernel(const uint4* __restrict__ k, const uint4* __restrict__ 
                          uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                          const int64_t* __restrict__ slot_mapping, int num_tokens,
                          int num_kv_heads, int64_t num_slots) {
+  // let a programmatic dependent (the attention kernel) get launched now; it
+  // waits for this grid's completion before reading the cache
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= (int64_t)num_tokens * num_kv_heads) return;
