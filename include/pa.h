@@ -80,14 +80,24 @@ int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_ca
 
 /*
  * Bytes of workspace pa_attention_varlen needs for a step of at most
- * num_seqs sequences, no sequence longer than max_seq_len tokens: fp32
- * split-K partials (running max, sum and unnormalised output per partition
- * of a sequence's keys) plus one int32 arrival counter per (sequence,
- * kv-head).  Always at least 256 for valid arguments; 0 means invalid
- * arguments.
+ * num_seqs sequences, no sequence longer than max_seq_len tokens: a status
+ * word, fp32 split-K partials (running max, sum and unnormalised output per
+ * partition of a sequence's keys), one int32 arrival counter per (sequence,
+ * kv-head) and the prefill work list.  0 means invalid arguments.
  */
 size_t pa_attention_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                    int head_dim, int max_seq_len);
+
+/*
+ * Read the workspace's status word (blocking: copies 4 bytes to *status_out
+ * and synchronises `stream`).  0 = every kernel of the previous calls ran to
+ * completion.  Bit 0 set = a kernel gave up waiting on one of its own
+ * pipeline barriers after a time limit instead of hanging (a library bug or a
+ * GPU fault); the outputs of that call are not valid.  The word stays set until
+ * pa_workspace_init clears the workspace again.
+ */
+int pa_workspace_status(const void* workspace, size_t workspace_bytes, int* status_out,
+                        struct CUstream_st* stream);
 
 /*
  * Zero a workspace before its first use (a cudaMemsetAsync on `stream`).
@@ -116,9 +126,10 @@ int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_s
  *   v_cache        [num_blocks][num_kv_heads][block_size][head_dim]
  *   block_tables   int32 [num_seqs][max_blocks_per_seq]; entries beyond
  *                  ceil(seq_lens[s] / block_size) are never read; an entry
- *                  outside [0, num_blocks) is never dereferenced (its keys
- *                  are left out of the softmax: the result is then not
- *                  meaningful, but no memory outside the pool is touched)
+ *                  outside [0, num_blocks) is never dereferenced (the result
+ *                  for that sequence is then not meaningful, but no memory
+ *                  outside the pool is touched).  Slots of the last block past
+ *                  seq_lens[s] are never used, whatever they hold.
  *   seq_lens       int32 [num_seqs]
  *   query_start_loc int32 [num_seqs + 1], query_start_loc[0] = 0,
  *                  nondecreasing, query_start_loc[num_seqs] = num_tokens

@@ -243,6 +243,19 @@ decode_splitk_kernel(const AttnParams p) {
       for (int u = 0; u < NV; ++u)
         vw[e][u] = lds128(vs + (tok * kChunks + ((8 * u + r) ^ v_swz(tok))) * 16);
     }
+    // slots of the last block past seq_len (and blocks outside the pool) may
+    // hold anything, NaN included: their V words become zeros so that the
+    // zero weights below cannot turn them into NaN in the P.V product
+    if (blk * kBlockSize + kBlockSize > L || !blk_ok) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = blk * kBlockSize + 2 * q4 + (e & 1) + 8 * (e >> 1);
+        if (!blk_ok || key >= L) {
+#pragma unroll
+          for (int u = 0; u < NV; ++u) vw[e][u] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
     // ---- scale, mask, online softmax
     const int key0 = blk * kBlockSize + 2 * q4;  // keys key0, +1 (half 0), key0+8, +9 (half 1)
     const bool tail = (blk * kBlockSize + kBlockSize > first_masked) || !blk_ok;

@@ -28,16 +28,23 @@ static int choose_part_tokens(int num_seqs, int num_kv_heads, int max_seq_len) {
   return part;
 }
 
-WorkspaceLayout workspace_layout(int num_seqs, int num_kv_heads, int head_dim, int max_seq_len) {
+WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int max_seq_len) {
   WorkspaceLayout w{};
   w.part_tokens = choose_part_tokens(num_seqs, num_kv_heads, max_seq_len);
   w.max_parts = max(1, (max_seq_len + w.part_tokens - 1) / w.part_tokens);
+  // prefill items: at most ceil(q_len / 128) <= ceil(max_seq_len / 128) per sequence and q-head
+  const long items = (long)num_seqs * ((max_seq_len + kPrefillQTile - 1) / kPrefillQTile) *
+                     num_q_heads;
+  w.max_items = (int)min(items, (long)(1 << 30));
   const size_t units = (size_t)num_seqs * num_kv_heads;
   const size_t slots = units * w.max_parts * kDecodeRows;
-  w.counter_off = 0;
-  w.o_off = align_up(units * sizeof(int), 256);
+  w.status_off = 0;
+  w.counter_off = 256;
+  w.o_off = align_up(w.counter_off + units * sizeof(int), 256);
   w.ml_off = align_up(w.o_off + slots * head_dim * sizeof(float), 256);
-  w.total = max((size_t)256, align_up(w.ml_off + slots * 2 * sizeof(float), 256));
+  w.items_off = align_up(w.ml_off + slots * 2 * sizeof(float), 256);
+  w.total = align_up(w.items_off + (size_t)(w.max_items + 1) * 16, 256);
   return w;
 }
 
@@ -81,7 +88,17 @@ extern "C" size_t pa_attention_workspace_size(int num_seqs, int num_q_heads, int
                                               int head_dim, int max_seq_len) {
   if (num_seqs < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_seq_len < 0) return 0;
   if (num_q_heads % num_kv_heads != 0 || !supported_head_dim(head_dim)) return 0;
-  return workspace_layout(num_seqs, num_kv_heads, head_dim, max_seq_len).total;
+  return workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len).total;
+}
+
+extern "C" int pa_workspace_status(const void* workspace, size_t workspace_bytes,
+                                   int* status_out, struct CUstream_st* stream) {
+  if (!workspace || workspace_bytes < 256 || !status_out) return PA_ERR_INVALID;
+  if (cudaMemcpyAsync(status_out, workspace, sizeof(int), cudaMemcpyDeviceToHost,
+                      (cudaStream_t)stream) != cudaSuccess ||
+      cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess)
+    return PA_ERR_CUDA;
+  return PA_OK;
 }
 
 extern "C" int pa_workspace_init(void* workspace, size_t workspace_bytes,
@@ -123,22 +140,30 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
 
   // ---- optional host copies: check the step and see which kernels it needs
   bool any_decode = true, any_prefill = true;
+  int prefill_items = -1;  // unknown without the host copies
   if (seq_lens_host && query_start_loc_host) {
     if (query_start_loc_host[0] != 0 || query_start_loc_host[num_seqs] != num_tokens)
       return PA_ERR_INVALID;
     any_decode = any_prefill = false;
+    prefill_items = 0;
     for (int s = 0; s < num_seqs; ++s) {
       const int ql = query_start_loc_host[s + 1] - query_start_loc_host[s];
       const int L = seq_lens_host[s];
       if (ql < 0 || ql > L || L > max_seq_len || ql > max_query_len) return PA_ERR_INVALID;
       if (ql == 0) continue;
-      if (ql * group <= kDecodeRows) any_decode = true; else any_prefill = true;
+      if (ql * group <= kDecodeRows) {
+        any_decode = true;
+      } else {
+        any_prefill = true;
+        prefill_items += (ql + kPrefillQTile - 1) / kPrefillQTile * num_q_heads;
+      }
     }
   } else if (max_query_len * group <= kDecodeRows) {
     any_prefill = false;
   }
 
-  const WorkspaceLayout w = workspace_layout(num_seqs, num_kv_heads, head_dim, max_seq_len);
+  const WorkspaceLayout w =
+      workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len);
   AttnParams p{};
   p.out = out;
   p.q = q;
@@ -165,17 +190,20 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
 
+  if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return PA_ERR_INVALID;
+  char* ws = (char*)workspace;
+  p.ws_status = (int*)(ws + w.status_off);
+  p.ws_counter = (int*)(ws + w.counter_off);
+  p.ws_o = (float*)(ws + w.o_off);
+  p.ws_ml = (float*)(ws + w.ml_off);
+  p.ws_items = (int4*)(ws + w.items_off);
+  p.max_items = w.max_items;
   if (any_decode) {
-    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return PA_ERR_INVALID;
-    char* ws = (char*)workspace;
-    p.ws_counter = (int*)(ws + w.counter_off);
-    p.ws_o = (float*)(ws + w.o_off);
-    p.ws_ml = (float*)(ws + w.ml_off);
     cudaError_t e = launch_decode_splitk(p, head_dim, max_query_len, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
   if (any_prefill) {
-    cudaError_t e = launch_attention_simple(p, head_dim, true, kDecodeRows, st);
+    cudaError_t e = launch_prefill_tcgen05(p, head_dim, max_query_len, prefill_items, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;

@@ -36,15 +36,24 @@ struct AttnParams {
   float* ws_o;       // [num_seqs*Hkv][max_parts][16][D] unnormalised partial outputs
   float* ws_ml;      // [num_seqs*Hkv][max_parts][16][2] running max (log2 units), sum
   int* ws_counter;   // [num_seqs*Hkv] arrival counters, zero between calls
+  // prefill work list
+  int* ws_status;    // [0]: error bits set by a kernel that gave up waiting; [1]: item count
+  int4* ws_items;    // prefill items (seq, q-tile, q-head, kv tiles)
+  int max_items;
 };
+
+// bits of ws_status[0]
+constexpr int kStatusWaitTimeout = 1;  // an mbarrier wait exceeded its time limit
 
 // Workspace layout shared by the size query and the launch.
 struct WorkspaceLayout {
   int part_tokens;
   int max_parts;
-  size_t counter_off, o_off, ml_off, total;
+  int max_items;
+  size_t status_off, counter_off, o_off, ml_off, items_off, total;
 };
-WorkspaceLayout workspace_layout(int num_seqs, int num_kv_heads, int head_dim, int max_seq_len);
+WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int max_seq_len);
 
 // Launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
@@ -60,5 +69,13 @@ cudaError_t launch_attention_simple(const AttnParams& p, int head_dim, bool is_b
 // Split-K decode kernel (bf16): sequences with q_len * group <= 16.
 cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
                                  cudaStream_t stream);
+
+// Tensor-core prefill kernel (bf16): sequences with q_len * group > 16.
+// num_items >= 0: the work list in ws_items was written by the host (exact
+// count); num_items < 0: build it on the device first.
+constexpr int kPrefillQTile = 128;  // query rows per work item (MMA M)
+constexpr int kPrefillKvTile = 128;  // keys per pipeline step
+cudaError_t launch_prefill_tcgen05(const AttnParams& p, int head_dim, int max_query_len,
+                                   int num_items, cudaStream_t stream);
 
 }  // namespace pa

@@ -20,7 +20,7 @@ PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
 
 # every symbol include/pa.h declares
 EXPORTS = ("pa_status_string", "pa_reshape_and_cache", "pa_attention_workspace_size",
-           "pa_workspace_init", "pa_attention_varlen")
+           "pa_workspace_init", "pa_workspace_status", "pa_attention_varlen")
 
 _lib = None
 
@@ -47,6 +47,8 @@ def library() -> ctypes.CDLL:
                                              c_int, c_int, c_p]
         lib.pa_attention_workspace_size.restype = c_sz
         lib.pa_attention_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int]
+        lib.pa_workspace_status.restype = c_int
+        lib.pa_workspace_status.argtypes = [c_p, c_sz, c_p, c_p]
         lib.pa_workspace_init.restype = c_int
         lib.pa_workspace_init.argtypes = [c_p, c_sz, c_p]
         lib.pa_attention_varlen.restype = c_int
@@ -118,6 +120,16 @@ def new_workspace(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: 
     if rc != PA_OK:
         raise PAError(rc, "pa_workspace_init")
     return ws
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Status word of a workspace (0 = every kernel so far ran to completion)."""
+    out = ctypes.c_int(0)
+    rc = library().pa_workspace_status(_dev(workspace, "workspace"), workspace.numel(),
+                                       ctypes.addressof(out), _stream(stream))
+    if rc != PA_OK:
+        raise PAError(rc, "pa_workspace_status")
+    return int(out.value)
 
 
 def attention_varlen(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,

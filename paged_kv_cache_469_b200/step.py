@@ -27,7 +27,7 @@ def to_torch(a: np.ndarray, device) -> torch.Tensor:
 
 class DeviceStep:
     def __init__(self, step: StepInputs, device: str = "cuda", *, max_blocks_per_seq=None,
-                 ctx_chunk_rows: int = 1 << 18):
+                 ctx_chunk_rows: int = 1 << 18, cache_fill: float = 0.0):
         self.step = step
         self.device = device
         plan = plan_step(free_queue=step.free_queue, seq_lens=step.seq_lens,
@@ -38,8 +38,10 @@ class DeviceStep:
         self.plan = plan
         dt = torch.float32 if step.dtype == "f32" else torch.bfloat16
         shape = (step.num_blocks, step.num_kv_heads, step.block_size, step.head_dim)
-        self.k_cache = torch.zeros(shape, dtype=dt, device=device)
-        self.v_cache = torch.zeros(shape, dtype=dt, device=device)
+        # cache_fill: what the never-written slots hold (a pool fresh from the
+        # allocator may hold anything; NaN is the worst case)
+        self.k_cache = torch.full(shape, cache_fill, dtype=dt, device=device)
+        self.v_cache = torch.full(shape, cache_fill, dtype=dt, device=device)
         # earlier tokens' K/V: written through the library, in chunks of rows
         n = step.k_ctx.shape[0]
         for s in range(0, n, ctx_chunk_rows):
