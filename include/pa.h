@@ -158,6 +158,43 @@ int pa_attention_varlen(void* out, const void* q, const void* k_cache, const voi
                         const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
                         struct CUstream_st* stream);
 
+/*
+ * pa_attention_varlen_static_scratch -- pa_attention_varlen for callers that
+ * cannot allocate device memory.  (The pages describe no such call; it has no
+ * counterpart in the method itself.)
+ *
+ * Who needs it: code that must not call cudaMalloc or any allocating routine
+ * -- a memory allocator's own callbacks (they would re-enter the allocator),
+ * a plugin whose host application owns every device buffer and passes it only
+ * inputs and outputs, or a latency-critical path where an allocation (which
+ * may synchronise the device) is not allowed.  Such a caller has nowhere to
+ * put the workspace pa_attention_varlen asks for.
+ *
+ * Same arguments and results as pa_attention_varlen, minus the workspace.
+ * The scratch instead lives in one fixed array of PA_STATIC_SCRATCH_BYTES
+ * (16 MiB) that every GPU which loads this library holds until the process
+ * exits.  A step whose pa_attention_workspace_size(...) exceeds that is
+ * rejected with PA_ERR_INVALID before anything is launched.  The call itself
+ * allocates nothing.
+ *
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call, on every stream, shares the one array and it keeps the last
+ *     call's contents: each call clears the parts that must start at zero.
+ *     Calls that can overlap on the GPU (other streams, other threads) race
+ *     on the array: serialise them.
+ *   - A kernel's status word (see pa_workspace_status) lives in this array
+ *     too and is cleared by the next call.
+ */
+#define PA_STATIC_SCRATCH_BYTES (16u << 20)
+int pa_attention_varlen_static_scratch(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+    const int32_t* query_start_loc, int num_seqs, int num_tokens, int max_query_len,
+    int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int num_blocks, float scale, pa_dtype dtype, const int32_t* seq_lens_host,
+    const int32_t* query_start_loc_host, struct CUstream_st* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,72 @@
+// pa_static_scratch.cu -- paged attention for callers that cannot allocate.
+//
+// pa_attention_varlen needs a caller-provided workspace.  Some callers have no
+// way to get one: code running inside a memory allocator's own callbacks (it
+// may not re-enter the allocator), plugins whose host application owns all
+// device memory and hands them only their inputs and outputs, and latency-
+// critical paths whose rules forbid a cudaMalloc (which can synchronise the
+// device and take milliseconds).  For them this file keeps a fixed scratch
+// area in a file-scope __device__ array, which the CUDA runtime places on
+// every GPU that loads the library when the module is loaded and keeps until
+// the process exits, and runs the same kernels on it.
+#include <mutex>
+
+#include "pa.h"
+#include "pa_internal.cuh"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_pa_scratch[PA_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_pa_scratch on the current device, looked up once per
+// device.  In host code the symbol names a host-side stand-in, never the
+// device array itself, so only this address may be handed to a kernel.
+int scratch_for_current_device(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_pa_scratch) != cudaSuccess || !ptr) return PA_ERR_CUDA;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_attention_varlen_static_scratch(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+    const int32_t* query_start_loc, int num_seqs, int num_tokens, int max_query_len,
+    int max_seq_len, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+    int num_blocks, float scale, pa_dtype dtype, const int32_t* seq_lens_host,
+    const int32_t* query_start_loc_host, struct CUstream_st* stream) {
+  const size_t need =
+      pa_attention_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len);
+  if (need == 0) return PA_ERR_INVALID;
+  if (need > (size_t)PA_STATIC_SCRATCH_BYTES) return PA_ERR_INVALID;  // step too large
+  void* scratch = nullptr;
+  const int rc = scratch_for_current_device(&scratch);
+  if (rc != PA_OK) return rc;
+  if (num_seqs > 0 && num_tokens > 0) {
+    // The array still holds whatever the previous call left there, possibly
+    // under another layout: the status word and the split-K arrival counters
+    // must start at zero, so clear them (everything before the partials).
+    const pa::WorkspaceLayout w =
+        pa::workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len);
+    if (cudaMemsetAsync(scratch, 0, w.o_off, (cudaStream_t)stream) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  return pa_attention_varlen(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                             query_start_loc, num_seqs, num_tokens, max_query_len, max_seq_len,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                             dtype, scratch, (size_t)PA_STATIC_SCRATCH_BYTES, seq_lens_host,
+                             query_start_loc_host, stream);
+}

@@ -20,7 +20,8 @@ PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
 
 # every symbol include/pa.h declares
 EXPORTS = ("pa_status_string", "pa_reshape_and_cache", "pa_attention_workspace_size",
-           "pa_workspace_init", "pa_workspace_status", "pa_attention_varlen")
+           "pa_workspace_init", "pa_workspace_status", "pa_attention_varlen",
+           "pa_attention_varlen_static_scratch")
 
 _lib = None
 

@@ -1,0 +1,88 @@
+"""pa_attention_varlen_static_scratch: the attention call for callers that
+cannot allocate device memory (allocator callbacks, plugins that are handed
+only their inputs and outputs, paths where a cudaMalloc is not allowed).  It
+keeps its scratch in a fixed array inside the library instead of a workspace
+from the caller.
+
+Its result must match pa_attention_varlen's on the same step, on two calls in
+a row (the second call finds the first call's leftovers in the shared array).
+This file is collected last so that a run stopping at the first failure has
+already run every other test."""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_469_b200 import lib
+from paged_kv_cache_469_b200.inputs import random_step
+from tests.test_gpu_parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
+
+
+def _entry():
+    f = lib.library().pa_attention_varlen_static_scratch
+    c_int, c_p, c_f = ctypes.c_int, ctypes.c_void_p, ctypes.c_float
+    f.restype = c_int
+    f.argtypes = [c_p, c_p, c_p, c_p, c_p, c_int, c_p, c_p, c_int, c_int, c_int, c_int, c_int,
+                  c_int, c_int, c_int, c_int, c_f, c_int, c_p, c_p, c_p]
+    return f
+
+
+def _call(f, ds, out):
+    p = ds.plan
+    sl = np.ascontiguousarray(p.seq_lens, np.int32)
+    qs = np.ascontiguousarray(p.query_start_loc, np.int32)
+    q = ds.q
+    return f(out.data_ptr(), q.data_ptr(), ds.k_cache.data_ptr(), ds.v_cache.data_ptr(),
+             ds.block_tables.data_ptr(), ds.block_tables.shape[1], ds.seq_lens.data_ptr(),
+             ds.query_start_loc.data_ptr(), len(sl), q.shape[0], p.max_query_len, p.max_seq_len,
+             q.shape[1], ds.k_cache.shape[1], q.shape[2], ds.k_cache.shape[2],
+             ds.k_cache.shape[0], float(ds.step.scale), lib.PA_DTYPE_BF16, sl.ctypes.data,
+             qs.ctypes.data, torch.cuda.current_stream().cuda_stream)
+
+
+def test_static_scratch_matches_workspace_call_twice():
+    from paged_kv_cache_469_b200.step import DeviceStep
+    f = _entry()
+    # two different steps (decode-class and prefill-class sequences, both head
+    # sizes), so the second call sees a different layout's leftovers
+    steps = [random_step(901, dtype="bf16", num_q_heads=16, num_kv_heads=4, head_dim=128,
+                         num_seqs=8, max_ctx=1500, max_q=150),
+             random_step(902, dtype="bf16", num_q_heads=32, num_kv_heads=4, head_dim=64,
+                         num_seqs=12, max_ctx=2500, max_q=3)]
+    for step in steps:
+        ds = DeviceStep(step)
+        need = lib.attention_workspace_size(step.num_seqs, step.num_q_heads, step.num_kv_heads,
+                                            step.head_dim, ds.plan.max_seq_len)
+        assert 0 < need <= STATIC_SCRATCH_BYTES
+        ds.run()  # the workspace path: cache write + pa_attention_varlen
+        torch.cuda.synchronize()
+        ref = ds.out.float().cpu().numpy().astype(np.float64)
+        for _ in range(2):
+            out = torch.full_like(ds.out, float("nan"))
+            assert _call(f, ds, out) == lib.PA_OK
+            torch.cuda.synchronize()
+            assert_close(out.float().cpu().numpy().astype(np.float64), ref, "bf16",
+                         "static-scratch call vs workspace call")
+
+
+def test_static_scratch_rejects_a_step_beyond_its_size():
+    f = _entry()
+    dev = "cuda"
+    kc = torch.zeros(4, 8, 16, 128, dtype=torch.bfloat16, device=dev)
+    q = torch.zeros(1, 32, 128, dtype=torch.bfloat16, device=dev)
+    bt = torch.zeros(1, 8192, dtype=torch.int32, device=dev)
+    sl = torch.ones(1, dtype=torch.int32, device=dev)
+    qs = torch.tensor([0, 1], dtype=torch.int32, device=dev)
+    big_seqs, big_len = 4096, 131072  # far more scratch than the fixed array holds
+    assert lib.attention_workspace_size(big_seqs, 32, 8, 128, big_len) > STATIC_SCRATCH_BYTES
+    rc = f(q.data_ptr(), q.data_ptr(), kc.data_ptr(), kc.data_ptr(), bt.data_ptr(), 8192,
+           sl.data_ptr(), qs.data_ptr(), big_seqs, 1, 1, big_len, 32, 8, 128, 16, 4, 0.1,
+           lib.PA_DTYPE_BF16, None, None, torch.cuda.current_stream().cuda_stream)
+    assert rc == lib.PA_ERR_INVALID
