@@ -5,11 +5,13 @@
 // bandwidth; section "PagedAttentionの仕組み": the keys are read block by
 // block through the sequence's block table.
 //
-// Work split.  One CTA (4 warps) per (partition of part_tokens keys, kv-head,
-// sequence).  All q-heads of the kv-head (and, for a short multi-token decode,
-// all its query tokens) form the rows of one 16-row MMA tile, so every K/V
-// byte is read from HBM once per kv-head.  Warp w of the CTA takes blocks
-// w, w+4, ... of the partition.
+// Work split.  One CTA (kWarps warps) per (partition of part_tokens keys,
+// kv-head, sequence); the hardware hands CTAs to SMs as they free up, which
+// balances the load even though SMs do not all get the same share of memory
+// bandwidth.  All q-heads of the kv-head (and, for a short multi-token
+// decode, all its query tokens) form the rows of one 16-row MMA tile, so every
+// K/V byte is read from HBM once per kv-head.  Warp w of the CTA takes blocks
+// w, w+kWarps, ... of the partition.
 //
 // Staging.  Each warp streams its blocks through a private ring of kStages
 // shared-memory slots (one (block, kv-head) K tile + V tile per slot) with
@@ -26,7 +28,7 @@
 // output's D axis is permuted so that every lane's V words are 8 consecutive
 // bf16 of one key row (undone when the output is stored).
 //
-// Split-K.  A CTA reduces its 4 warps' (max, sum, O) in shared memory.  A
+// Split-K.  A CTA reduces its warps' (max, sum, O) in shared memory.  A
 // sequence that fits one partition writes its output directly; otherwise each
 // partition stores its fp32 partial in the workspace and bumps a per
 // (sequence, kv-head) counter; the CTA that arrives last merges all partials
@@ -38,6 +40,14 @@
 #include <math.h>
 
 #include "pa_internal.cuh"
+
+// ring slots per warp (shared memory per CTA: warps x stages x 2 tiles)
+#ifndef PA_DECODE_STAGES_D64
+#define PA_DECODE_STAGES_D64 4
+#endif
+#ifndef PA_DECODE_STAGES_D128
+#define PA_DECODE_STAGES_D128 3
+#endif
 
 namespace pa {
 namespace {
@@ -101,8 +111,8 @@ struct DecodeSmem {
   static constexpr int kSlotBytes = 2 * kTileBytes;      // K tile + V tile
 };
 
-template <int D, bool kRows16, int kStages>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+template <int D, bool kRows16, int kStages, int kWarps>
+__global__ void __launch_bounds__(kWarps * 32)
 decode_splitk_kernel(const AttnParams p) {
   constexpr int NJ = D / 32;  // 16-byte K chunks per key row a lane reads
   constexpr int NV = D / 64;  // 16-byte V chunks per key row a lane reads
@@ -113,8 +123,8 @@ decode_splitk_kernel(const AttnParams p) {
   constexpr int kCopies = kBlockSize * kChunks / 32;  // 16-byte copies per lane per tile
 
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ float sh_m[kDecodeWarps][kDecodeRows];
-  __shared__ float sh_l[kDecodeWarps][kDecodeRows];
+  __shared__ float sh_m[kWarps][kDecodeRows];
+  __shared__ float sh_l[kWarps][kDecodeRows];
   __shared__ int sh_last;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -136,7 +146,7 @@ decode_splitk_kernel(const AttnParams p) {
   const int nparts = (L + P - 1) / P;
   // a sequence longer than the bounds the workspace was sized for is left
   // unwritten rather than overrunning the workspace or its block-table row
-  if (part >= nparts || nparts > p.max_parts ||
+  if (part >= nparts || nparts > p.max_parts || L > p.max_seq_len ||
       (L + kBlockSize - 1) / kBlockSize > p.max_blocks_per_seq)
     return;
   const int t_begin = part * P;
@@ -146,9 +156,17 @@ decode_splitk_kernel(const AttnParams p) {
 
   // ---- this warp's block ids, one per lane (lane i <-> i-th block of the warp)
   const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
-  const int my_nblk = (blk_end - blk_begin - warp + kDecodeWarps - 1) / kDecodeWarps;
-  int my_id = 0;
-  if (lane < my_nblk) my_id = table[blk_begin + warp + kDecodeWarps * lane];
+  const int my_nblk = (blk_end - blk_begin - warp + kWarps - 1) / kWarps;
+  int win = -1, win_id = 0;  // block ids of the warp's blocks 32*win .. 32*win+31
+  auto block_id = [&](int i) {
+    if ((i >> 5) != win) {
+      win = i >> 5;
+      const int ii = (win << 5) + lane;
+      win_id = ii < my_nblk ? table[blk_begin + warp + kWarps * ii] : 0;
+    }
+    return __shfl_sync(0xffffffffu, win_id, i & 31);
+  };
+  uint32_t bad = 0;  // bit (slot): that slot's block id was outside the pool
 
   // ---- Q as the A operand (rows r and r+8), D axis permuted as the K chunks
   const __nv_bfloat16* qg = (const __nv_bfloat16*)p.q;
@@ -180,8 +198,13 @@ decode_splitk_kernel(const AttnParams p) {
                         warp * kStages * SM::kSlotBytes;
 
   auto issue = [&](int i) {  // copy the warp's i-th block into slot i % kStages
-    int id = __shfl_sync(0xffffffffu, my_id, i);
-    if (id < 0 || id >= p.num_blocks) id = 0;  // never dereference outside the pool
+    int id = block_id(i);
+    if (id < 0 || id >= p.num_blocks) {  // never dereference outside the pool
+      id = 0;
+      bad |= 1u << (i % kStages);
+    } else {
+      bad &= ~(1u << (i % kStages));
+    }
     const char* kt = kc + id * blk_bytes + head_off;
     const char* vt = vc + id * blk_bytes + head_off;
     const uint32_t ks = ring + (i % kStages) * SM::kSlotBytes;
@@ -213,9 +236,8 @@ decode_splitk_kernel(const AttnParams p) {
     cp_async_wait<kStages - 1>();  // this lane's copies of block i have landed
     __syncwarp();                  // ... and every other lane's
 
-    const int blk = blk_begin + warp + kDecodeWarps * i;
-    const int id_raw = __shfl_sync(0xffffffffu, my_id, i);
-    const bool blk_ok = id_raw >= 0 && id_raw < p.num_blocks;
+    const int blk = blk_begin + warp + kWarps * i;
+    const bool blk_ok = !((bad >> (i % kStages)) & 1u);
     const uint32_t ks = ring + (i % kStages) * SM::kSlotBytes;
     const uint32_t vs = ks + SM::kTileBytes;
 
@@ -339,7 +361,7 @@ decode_splitk_kernel(const AttnParams p) {
   }
   __syncthreads();
 
-  // ---- merge the 4 warps: row-wise max, rescaled sums
+  // ---- merge the warps: row-wise max, rescaled sums
   const int unit = s * p.num_kv_heads + kvh;
   const bool direct = (nparts == 1);
   __nv_bfloat16* out = (__nv_bfloat16*)p.out;
@@ -347,11 +369,11 @@ decode_splitk_kernel(const AttnParams p) {
     const int row = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sh_m[w][row]);
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sh_m[w][row]);
     const float base = (M == -INFINITY) ? 0.f : M;
     float Ls = 0.f, Os = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
       const float f = exp2f(sh_m[w][row] - base);
       Ls += sh_l[w][row] * f;
       Os += sh_o[w][row][d] * f;
@@ -401,15 +423,16 @@ decode_splitk_kernel(const AttnParams p) {
 
 template <int D, bool kRows16, int kStages>
 cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
-  auto kernel = decode_splitk_kernel<D, kRows16, kStages>;
-  const int ring = kDecodeWarps * kStages * DecodeSmem<D>::kSlotBytes;
-  const int merge = kDecodeWarps * kDecodeRows * D * (int)sizeof(float);
+  constexpr int kWarps = kDecodeWarps;
+  auto kernel = decode_splitk_kernel<D, kRows16, kStages, kWarps>;
+  const int ring = kWarps * kStages * DecodeSmem<D>::kSlotBytes;
+  const int merge = kWarps * kDecodeRows * D * (int)sizeof(float);
   const int smem = ring > merge ? ring : merge;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.max_parts, p.num_kv_heads, p.num_seqs);
-  cfg.blockDim = dim3(kDecodeWarps * 32);
+  cfg.blockDim = dim3(kWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -428,10 +451,11 @@ cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_quer
   const int max_rows = min(max_query_len * p.group, kDecodeRows);
   const bool rows16 = max_rows > 8;
   cudaError_t e;
+  constexpr int s64 = PA_DECODE_STAGES_D64, s128 = PA_DECODE_STAGES_D128;
   if (head_dim == 64)
-    e = rows16 ? launch_one<64, true, 4>(p, stream) : launch_one<64, false, 4>(p, stream);
+    e = rows16 ? launch_one<64, true, s64>(p, stream) : launch_one<64, false, s64>(p, stream);
   else
-    e = rows16 ? launch_one<128, true, 3>(p, stream) : launch_one<128, false, 3>(p, stream);
+    e = rows16 ? launch_one<128, true, s128>(p, stream) : launch_one<128, false, s128>(p, stream);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -9,21 +9,24 @@ namespace pa {
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Keys per split-K partition: the largest power of two in [256, 2048] that
-// still gives the GPU about eight waves' worth of CTAs when sequences average
-// half of max_seq_len.  (2048 = 4 warps x 32 blocks: each lane of a warp holds
-// one block id of the partition.)
+// Keys per split-K partition: the largest power of two in [PA_PART_MIN,
+// PA_PART_MAX] that still gives the GPU about PA_TARGET_CTAS CTAs when the
+// sequences average half of max_seq_len.  Hardware CTA scheduling then spreads
+// the partitions over the SMs as they free up.
 #ifndef PA_PART_MIN
-#define PA_PART_MIN 512
+#define PA_PART_MIN 1024
+#endif
+#ifndef PA_PART_MAX
+#define PA_PART_MAX 2048
 #endif
 #ifndef PA_TARGET_CTAS
 #define PA_TARGET_CTAS (8 * 148)
 #endif
 static int choose_part_tokens(int num_seqs, int num_kv_heads, int max_seq_len) {
   const long units = (long)num_seqs * num_kv_heads;
-  const long target = PA_TARGET_CTAS;
-  int part = 2048;
-  while (part > PA_PART_MIN && units * (((long)max_seq_len / 2 + part - 1) / part) < target)
+  int part = PA_PART_MAX;
+  while (part > PA_PART_MIN &&
+         units * (((long)max_seq_len / 2 + part - 1) / part) < (long)PA_TARGET_CTAS)
     part /= 2;
   return part;
 }
@@ -173,6 +176,9 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
   p.seq_lens = seq_lens;
   p.query_start_loc = query_start_loc;
   p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_seq_len = max_seq_len;
+  p.part_tokens = w.part_tokens;
+  p.max_parts = w.max_parts;
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;
   p.num_q_heads = num_q_heads;
@@ -181,8 +187,6 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
   p.num_blocks = num_blocks;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.part_tokens = w.part_tokens;
-  p.max_parts = w.max_parts;
   cudaStream_t st = (cudaStream_t)stream;
 
   if (dtype == PA_DTYPE_F32) {

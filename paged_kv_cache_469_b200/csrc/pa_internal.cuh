@@ -10,7 +10,10 @@ namespace pa {
 
 constexpr int kBlockSize = 16;       // tokens per cache block (the pages' default)
 constexpr int kDecodeRows = 16;      // query rows per kv-head one decode CTA holds (MMA M)
-constexpr int kDecodeWarps = 4;      // warps of a decode CTA
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+constexpr int kDecodeWarps = PA_DECODE_WARPS;  // warps of a decode CTA
 
 // Everything one attention launch reads; the same struct serves every kernel.
 struct AttnParams {
@@ -22,6 +25,7 @@ struct AttnParams {
   const int32_t* seq_lens;
   const int32_t* query_start_loc;
   int max_blocks_per_seq;
+  int max_seq_len;  // host bound: longer sequences are caller error and left unwritten
   int num_seqs;
   int num_tokens;
   int num_q_heads;
@@ -37,7 +41,7 @@ struct AttnParams {
   float* ws_ml;      // [num_seqs*Hkv][max_parts][16][2] running max (log2 units), sum
   int* ws_counter;   // [num_seqs*Hkv] arrival counters, zero between calls
   // prefill work list
-  int* ws_status;    // [0]: error bits set by a kernel that gave up waiting; [1]: item count
+  int* ws_status;    // [0]: error bits set by a kernel that gave up waiting
   int4* ws_items;    // prefill items (seq, q-tile, q-head, kv tiles)
   int max_items;
 };
