@@ -77,7 +77,7 @@ cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_quer
 // Tensor-core prefill kernel (bf16): sequences with q_len * group > 16.
 // num_items >= 0: the work list in ws_items was written by the host (exact
 // count); num_items < 0: build it on the device first.
-constexpr int kPrefillQTile = 128;  // query rows per work item (MMA M)
+constexpr int kPrefillQTile = 128;  // query rows per Q tile (MMA M); a work item holds two
 constexpr int kPrefillKvTile = 128;  // keys per pipeline step
 cudaError_t launch_prefill_tcgen05(const AttnParams& p, int head_dim, int max_query_len,
                                    int num_items, cudaStream_t stream);

@@ -10,16 +10,18 @@
 // Work item = (sequence, 128-query tile, q-head).  A persistent CTA walks its
 // items; per item it streams the sequence's keys in 128-key tiles:
 //
-//   warp 0      TMA producer: Q tile once per item, then K and V tiles, each
-//               tile eight 16-token cache blocks (one 16 x 64 box per block and
-//               64-wide slice of D, 128-byte swizzled, straight from the pool
-//               through the block table)
+//   warps 8, 10 TMA producers (warp 8: the two Q tiles once per item, then K
+//               tiles; warp 10: V tiles), each tile eight 16-token cache
+//               blocks (one 16 x 64 box per block and 64-wide slice of D,
+//               128-byte swizzled, straight from the pool through the block
+//               table)
 //   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (tcgen05.mma,
 //               M=128, N=128, K=16 steps), then O += P V into TMEM
 //   warps 2..5  softmax: one query row per thread; S from TMEM (tcgen05.ld),
 //               causal mask, online softmax in fp32 (exp2, the running max is
 //               only moved when it grows by more than 2^8, so O is rarely
-//               rescaled), P as bf16 into shared memory for the second MMA;
+//               rescaled), P as bf16 into shared memory (double-buffered) for
+//               the second MMA;
 //               at the end of the item O / l from TMEM to global memory
 //
 // S is double-buffered in TMEM so that Q K^T of tile j+1 overlaps the softmax
@@ -39,29 +41,39 @@
 namespace pa {
 namespace {
 
-constexpr int QT = kPrefillQTile;               // 128 query rows per item
-constexpr int KT = kPrefillKvTile;              // 128 keys per tile
+constexpr int QT = kPrefillQTile;               // 128 query rows per Q tile
+constexpr int KT = kPrefillKvTile;              // 128 keys per K/V tile
 constexpr int kTileBlocks = KT / kBlockSize;    // 8 cache blocks per tile
 constexpr int kKStages = 2, kVStages = 2;
-constexpr int kThreads = 192;                   // 6 warps
+constexpr int kThreads = 384;                   // 12 warps = 3 warpgroups
+// warpgroup 0 (warps 0..3): softmax of half 0; warpgroup 1 (4..7): softmax of
+// half 1 (a warp reads the TMEM lanes 32 * (warp % 4) ..); warpgroup 2: warp
+// 8 TMA for Q and K, warp 9 MMA issuer, warp 10 TMA for V, warp 11 idle.
+constexpr int kWarpK = 8, kWarpMma = 9, kWarpV = 10;
+// Registers: launched at 168 each (384 x 168 = 64512); warpgroup 2 then gives
+// back down to 88 and the softmax warpgroups take up to 208:
+// 2 x 128 x 208 + 128 x 88 = 64512.
+constexpr int kRegsLaunch = 168, kRegsSoftmax = 208, kRegsOther = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 0;                  // S buffers at columns 0 and 128
-constexpr uint32_t kTmemO = 256;                // O at columns 256 .. 256+D
+// TMEM columns: O of half h at 128 h; S of half h at 256 + 128 h, its P (bf16,
+// two per column) written over the first 64 columns of S once S is read
+constexpr uint32_t kTmemO = 0, kTmemS = 256;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: move the max only past 2^8
 
 template <int D>
 struct PrefillLayout {
   static constexpr int kPanels = D / 64;            // 64-wide slices of D
-  static constexpr int kPanelBytes = 128 * 128;     // 128 rows x 128 bytes
-  static constexpr int kQBytes = kPanels * kPanelBytes;
-  static constexpr int kKvBytes = kPanels * kPanelBytes;
-  static constexpr int kPBytes = 2 * kPanelBytes;   // 128 rows x 128 keys bf16
-  static constexpr int q_off = 0;
-  static constexpr int k_off = q_off + kQBytes;
+  static constexpr int kQPanelBytes = QT * 128;     // 128 rows x 128 bytes
+  static constexpr int kKvPanelBytes = KT * 128;    // 128 rows x 128 bytes
+  static constexpr int kQBytes = kPanels * kQPanelBytes;   // one Q tile
+  static constexpr int kKvBytes = kPanels * kKvPanelBytes; // one K or V tile
+  static constexpr int q_off = 0;                   // two Q tiles (the two halves)
+  static constexpr int k_off = q_off + 2 * kQBytes;
   static constexpr int v_off = k_off + kKStages * kKvBytes;
-  static constexpr int p_off = v_off + kVStages * kKvBytes;
-  static constexpr int bar_off = p_off + kPBytes;
+  static constexpr int bar_off = v_off + kVStages * kKvBytes;
   static constexpr int used = bar_off + 256;
   // D = 64 would fit two CTAs per SM, whose TMEM allocations would then queue
   // behind each other: ask for enough shared memory to keep one CTA per SM.
@@ -70,9 +82,17 @@ struct PrefillLayout {
 
 // mbarrier indices
 enum : int {
-  kBarQFull = 0, kBarQEmpty, kBarKFull0, kBarKFull1, kBarKEmpty0, kBarKEmpty1, kBarVFull0,
-  kBarVFull1, kBarVEmpty0, kBarVEmpty1, kBarSFull0, kBarSFull1, kBarPFull, kBarODone, kNumBars
+  kBarQFull = 0, kBarQEmpty,
+  kBarKFull = 2,                      // + stage
+  kBarKEmpty = kBarKFull + kKStages,  // + stage
+  kBarVFull = kBarKEmpty + kKStages,  // + stage
+  kBarVEmpty = kBarVFull + kVStages,  // + stage
+  kBarSFull = kBarVEmpty + kVStages,  // + half
+  kBarPFull = kBarSFull + 2,          // + half
+  kBarODone = kBarPFull + 2,          // + half
+  kNumBars = kBarODone + 2
 };
+static_assert(kNumBars * 8 <= 256, "barriers must fit their 256-byte area");
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -158,6 +178,15 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// the same, with A (M x 16, bf16 packed two per 32-bit column) read from TMEM
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -240,15 +269,17 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, int a_mn_major, 
          ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// A work item is two 128-row Q tiles that read the same keys: two q-heads of
+// one kv-head (pair_heads), or two consecutive query tiles of one q-head.
 struct ItemInfo {
-  int seq, qtile, head, ntiles;
+  int seq, qt0, head0, ntiles;
   int q0, ql, L;
 };
 
 __device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int w) {
   const int4 it = p.ws_items[1 + w];
   ItemInfo r;
-  r.seq = it.x; r.qtile = it.y; r.head = it.z; r.ntiles = it.w;
+  r.seq = it.x; r.qt0 = it.y; r.head0 = it.z; r.ntiles = it.w;
   r.q0 = p.query_start_loc[r.seq];
   r.ql = p.query_start_loc[r.seq + 1] - r.q0;
   r.L = p.seq_lens[r.seq];
@@ -265,7 +296,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v) {
+                       const __grid_constant__ CUtensorMap tm_v, int pair_heads) {
   using LY = PrefillLayout<D>;
   constexpr int kPanels = LY::kPanels;
   extern __shared__ unsigned char smem_raw[];
@@ -275,7 +306,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = ((uint32_t)__cvta_generic_to_shared(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = base + LY::q_off, sK = base + LY::k_off, sV = base + LY::v_off,
-                 sP = base + LY::p_off, sBar = base + LY::bar_off;
+                 sBar = base + LY::bar_off;
   auto bar = [&](int i) { return sBar + 8u * (uint32_t)i; };
   volatile int* abort_flag = &sh_abort;
 
@@ -283,21 +314,25 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     sh_abort = 0;
     mbar_init(bar(kBarQFull), 1);
     mbar_init(bar(kBarQEmpty), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarKFull0 + i), 1);
-      mbar_init(bar(kBarKEmpty0 + i), 1);
-      mbar_init(bar(kBarVFull0 + i), 1);
-      mbar_init(bar(kBarVEmpty0 + i), 1);
-      mbar_init(bar(kBarSFull0 + i), 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(bar(kBarKFull + i), 1);
+      mbar_init(bar(kBarKEmpty + i), 1);
     }
-    mbar_init(bar(kBarPFull), 4);  // one arrival per softmax warp
-    mbar_init(bar(kBarODone), 1);
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(bar(kBarVFull + i), 1);
+      mbar_init(bar(kBarVEmpty + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarPFull + i), 4);  // one arrival per softmax warp of the half
+      mbar_init(bar(kBarODone + i), 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc((uint32_t)__cvta_generic_to_shared(&sh_tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -311,126 +346,161 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   const int num_items = p.ws_items[0].x;
   int* status = p.ws_status;
 
-  if (warp == 0) {
-    // =========================== TMA producer ===========================
-    const int oob_bh = p.num_blocks * p.num_kv_heads;  // first block-head row past the pool
-    uint32_t g = 0;                                     // global tile counter
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int w = item_index(k);
-      if (w >= num_items) break;
-      const ItemInfo it = load_item(p, w);
-      const int kvh = it.head / p.group;
-      const int nblk = (it.L + kBlockSize - 1) / kBlockSize;
-      const int shift = nblk * kBlockSize - it.L;  // unwritten slots of the last block
-      const int32_t* table = p.block_tables + (int64_t)it.seq * p.max_blocks_per_seq;
-      // ---- Q tile
-      if (lane == 0) {
-        if (k > 0) ok = wait_bar(bar(kBarQEmpty), (k - 1) & 1, abort_flag, status);
-        if (ok) {
-          mbar_expect_tx(bar(kBarQFull), LY::kQBytes);
-          for (int pn = 0; pn < kPanels; ++pn)
-            tma_load_3d(sQ + pn * LY::kPanelBytes, &tm_q, 64 * pn, it.head,
-                        it.q0 + it.qtile * QT, bar(kBarQFull));
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      // ---- K and V tiles
-      for (int t = 0; t < it.ntiles && ok; ++t, ++g) {
-        int id = -1;
-        const int lb = t * kTileBlocks + lane;
-        if (lane < kTileBlocks && lb < nblk && lb < p.max_blocks_per_seq) id = table[lb];
-        int c1[kTileBlocks], c2[kTileBlocks];
-#pragma unroll
-        for (int b = 0; b < kTileBlocks; ++b) {
-          const int idb = __shfl_sync(0xffffffffu, id, b);
-          const int lbb = t * kTileBlocks + b;
-          const bool valid = lbb < nblk && idb >= 0 && idb < p.num_blocks;
-          c1[b] = (valid && lbb == nblk - 1) ? -shift : 0;
-          c2[b] = valid ? idb * p.num_kv_heads + kvh : oob_bh;
-        }
-        if (lane == 0) {
-          const int ks = g % kKStages, vs = g % kVStages;
-          if (g >= kKStages)
-            ok = wait_bar(bar(kBarKEmpty0 + ks), ((g / kKStages) - 1) & 1, abort_flag, status);
+  if (warp >= 8) {
+    // warpgroup 2 gives registers back before taking its role
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    if (warp == kWarpK || warp == kWarpV) {
+      // ============ TMA producers: one warp loads the Q tiles and K, one loads V ============
+      // (separate warps, so that a K tile never waits behind a V slot)
+      const bool is_v = (warp == kWarpV);
+      const int oob_bh = p.num_blocks * p.num_kv_heads;  // first block-head row past the pool
+      uint32_t g = 0;                                     // global tile counter
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int w = item_index(k);
+        if (w >= num_items) break;
+        const ItemInfo it = load_item(p, w);
+        const int kvh = it.head0 / p.group;
+        const int nblk = (it.L + kBlockSize - 1) / kBlockSize;
+        const int shift = nblk * kBlockSize - it.L;  // unwritten slots of the last block
+        const int32_t* table = p.block_tables + (int64_t)it.seq * p.max_blocks_per_seq;
+        // ---- the two Q tiles
+        if (!is_v && lane == 0) {
+          if (k > 0) ok = wait_bar(bar(kBarQEmpty), (k - 1) & 1, abort_flag, status);
           if (ok) {
-            mbar_expect_tx(bar(kBarKFull0 + ks), LY::kKvBytes);
-            for (int pn = 0; pn < kPanels; ++pn)
-              for (int b = 0; b < kTileBlocks; ++b)
-                tma_load_3d(sK + ks * LY::kKvBytes + pn * LY::kPanelBytes + b * 2048, &tm_k,
-                            64 * pn, c1[b], c2[b], bar(kBarKFull0 + ks));
-          }
-          if (ok && g >= kVStages)
-            ok = wait_bar(bar(kBarVEmpty0 + vs), ((g / kVStages) - 1) & 1, abort_flag, status);
-          if (ok) {
-            mbar_expect_tx(bar(kBarVFull0 + vs), LY::kKvBytes);
-            for (int pn = 0; pn < kPanels; ++pn)
-              for (int b = 0; b < kTileBlocks; ++b)
-                tma_load_3d(sV + vs * LY::kKvBytes + pn * LY::kPanelBytes + b * 2048, &tm_v,
-                            64 * pn, c1[b], c2[b], bar(kBarVFull0 + vs));
+            mbar_expect_tx(bar(kBarQFull), 2 * LY::kQBytes);
+            for (int h = 0; h < 2; ++h) {
+              const int head = pair_heads ? it.head0 + h : it.head0;
+              const int qt = pair_heads ? it.qt0 : it.qt0 + h;
+              for (int pn = 0; pn < kPanels; ++pn)
+                tma_load_3d(sQ + h * LY::kQBytes + pn * LY::kQPanelBytes, &tm_q, 64 * pn, head,
+                            it.q0 + qt * QT, bar(kBarQFull));
+            }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-      }
-    }
-  } else if (warp == 1) {
-    // =========================== MMA issuer ===========================
-    constexpr uint32_t idesc_qk = instr_desc(128, KT, 0, 0);
-    constexpr uint32_t idesc_pv = instr_desc(128, D, 0, 1);
-    uint32_t g = 0;
-    bool ok = true;
-    auto issue_pv = [&](uint32_t gt, bool first_of_item) {
-      const int vs = gt % kVStages;
-      ok = wait_bar(bar(kBarPFull), gt & 1, abort_flag, status) &&
-           wait_bar(bar(kBarVFull0 + vs), (gt / kVStages) & 1, abort_flag, status);
-      if (!ok) return;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t vbase = sV + vs * LY::kKvBytes;
-#pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk) {
-          const uint64_t a = smem_desc(sP + (kk / 4) * LY::kPanelBytes + (kk % 4) * 32, 16, 1024);
-          const uint64_t b = smem_desc(vbase + kk * 2048, LY::kPanelBytes, 1024);
-          umma_bf16(tmem + kTmemO, a, b, idesc_pv, (first_of_item && kk == 0) ? 0u : 1u);
+        // ---- K or V tiles
+        for (int t = 0; t < it.ntiles && ok; ++t, ++g) {
+          int id = -1;
+          const int lb = t * kTileBlocks + lane;
+          if (lane < kTileBlocks && lb < nblk && lb < p.max_blocks_per_seq) id = table[lb];
+          int c1[kTileBlocks], c2[kTileBlocks];
+  #pragma unroll
+          for (int b = 0; b < kTileBlocks; ++b) {
+            const int idb = __shfl_sync(0xffffffffu, id, b);
+            const int lbb = t * kTileBlocks + b;
+            const bool valid = lbb < nblk && idb >= 0 && idb < p.num_blocks;
+            c1[b] = (valid && lbb == nblk - 1) ? -shift : 0;
+            c2[b] = valid ? idb * p.num_kv_heads + kvh : oob_bh;
+          }
+          if (lane == 0) {
+            const uint32_t nst = is_v ? kVStages : kKStages;
+            const int st = g % nst;
+            const int full = (is_v ? kBarVFull : kBarKFull) + st;
+            const int empty = (is_v ? kBarVEmpty : kBarKEmpty) + st;
+            const uint32_t dst = (is_v ? sV : sK) + st * LY::kKvBytes;
+            const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+            if (g >= nst) ok = wait_bar(bar(empty), ((g / nst) - 1) & 1, abort_flag, status);
+            if (ok) {
+              mbar_expect_tx(bar(full), LY::kKvBytes);
+              for (int pn = 0; pn < kPanels; ++pn)
+                for (int b = 0; b < kTileBlocks; ++b)
+                  tma_load_3d(dst + pn * LY::kKvPanelBytes + b * 2048, map, 64 * pn, c1[b], c2[b],
+                              bar(full));
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
         }
-        umma_commit(bar(kBarVEmpty0 + vs));
-        umma_commit(bar(kBarODone));
       }
-      __syncwarp();
-    };
-    for (int k = 0; ok; ++k) {
-      const int w = item_index(k);
-      if (w >= num_items) break;
-      const ItemInfo it = load_item(p, w);
-      ok = wait_bar(bar(kBarQFull), k & 1, abort_flag, status);
-      const uint32_t g_first = g;
-      for (int t = 0; t < it.ntiles && ok; ++t, ++g) {
-        const int ks = g % kKStages;
-        ok = wait_bar(bar(kBarKFull0 + ks), (g / kKStages) & 1, abort_flag, status);
-        if (!ok) break;
+    } else if (warp == kWarpMma) {
+      // =========================== MMA issuer ===========================
+      // Per half h: S_h = Q_h K^T (both operands in shared memory), then, once
+      // the softmax has written P_h over S_h in TMEM, O_h += P_h V (P from TMEM).
+      // The tensor pipe runs a thread's MMAs in order, so P.V of tile g-1 has
+      // finished with P_h before Q K^T of tile g overwrites S_h.
+      // Descriptors are built once; a k-step, panel or stage moves the start
+      // address, i.e. adds (byte offset >> 4) to the descriptor.
+      constexpr uint32_t idesc_qk = instr_desc(128, KT, 0, 0);
+      constexpr uint32_t idesc_pv = instr_desc(128, D, 0, 1);
+      const uint64_t dq0 = smem_desc(sQ, 16, 1024);
+      const uint64_t dk0 = smem_desc(sK, 16, 1024);
+      const uint64_t dv0 = smem_desc(sV, LY::kKvPanelBytes, 1024);
+      uint32_t g = 0;
+      bool ok = true;
+      auto issue_pv = [&](int h, uint32_t gt, bool first_of_item) {  // O_h += P_h V (tile gt)
+        ok = wait_bar(bar(kBarPFull + h), gt & 1, abort_flag, status);
+        if (!ok) return;
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t kbase = sK + ks * LY::kKvBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * LY::kPanelBytes + (kk % 4) * 32;
-            umma_bf16(tmem + kTmemS + (g & 1) * KT, smem_desc(sQ + off, 16, 1024),
-                      smem_desc(kbase + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(bar(kBarKEmpty0 + ks));
-          umma_commit(bar(kBarSFull0 + (g & 1)));
-          if (t == it.ntiles - 1) umma_commit(bar(kBarQEmpty));
+          const uint64_t dv = dv0 + (uint64_t)(((gt % kVStages) * LY::kKvBytes) >> 4);
+          const uint32_t dst = tmem + kTmemO + 128 * h;
+          const uint32_t pa = tmem + kTmemS + 128 * h;
+  #pragma unroll
+          for (int kk = 0; kk < KT / 16; ++kk)
+            umma_bf16_ts(dst, pa + 8 * kk, dv + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                         (first_of_item && kk == 0) ? 0u : 1u);
+          umma_commit(bar(kBarODone + h));
         }
         __syncwarp();
-        if (t > 0) issue_pv(g - 1, g - 1 == g_first);
+      };
+      auto issue_qk = [&](int h, uint32_t gt) {  // S_h = Q_h K^T (tile gt)
+        if (lane == 0) {
+          const uint64_t dk = dk0 + (uint64_t)(((gt % kKStages) * LY::kKvBytes) >> 4);
+          const uint64_t dq = dq0 + (uint64_t)((h * LY::kQBytes) >> 4);
+          const uint32_t dst = tmem + kTmemS + 128 * h;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qo = ((kk / 4) * LY::kQPanelBytes + (kk % 4) * 32) >> 4;
+            const uint32_t ko = ((kk / 4) * LY::kKvPanelBytes + (kk % 4) * 32) >> 4;
+            umma_bf16(dst, dq + qo, dk + ko, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(kBarSFull + h));
+        }
+        __syncwarp();
+      };
+      for (int k = 0; ok; ++k) {
+        const int w = item_index(k);
+        if (w >= num_items) break;
+        const ItemInfo it = load_item(p, w);
+        ok = wait_bar(bar(kBarQFull), k & 1, abort_flag, status);
+        const uint32_t g_first = g;
+        for (int t = 0; t < it.ntiles && ok; ++t, ++g) {
+          ok = wait_bar(bar(kBarKFull + g % kKStages), (g / kKStages) & 1, abort_flag, status);
+          if (ok && t > 0)
+            ok = wait_bar(bar(kBarVFull + (g - 1) % kVStages), ((g - 1) / kVStages) & 1, abort_flag,
+                          status);
+          if (!ok) break;
+          tc_fence_after();
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (t > 0) issue_pv(h, g - 1, g - 1 == g_first);  // P_h of the previous tile
+            if (ok) issue_qk(h, g);
+          }
+          if (ok && lane == 0) {
+            umma_commit(bar(kBarKEmpty + g % kKStages));
+            if (t > 0) umma_commit(bar(kBarVEmpty + (g - 1) % kVStages));
+            if (t == it.ntiles - 1) umma_commit(bar(kBarQEmpty));
+          }
+          __syncwarp();
+        }
+        if (ok && it.ntiles > 0) {  // P.V of the item's last tile
+          const uint32_t gl = g - 1;
+          ok = wait_bar(bar(kBarVFull + gl % kVStages), (gl / kVStages) & 1, abort_flag, status);
+          if (ok) tc_fence_after();
+          for (int h = 0; h < 2 && ok; ++h) issue_pv(h, gl, gl == g_first);
+          if (ok && lane == 0) umma_commit(bar(kBarVEmpty + gl % kVStages));
+          __syncwarp();
+        }
       }
-      if (ok && it.ntiles > 0) issue_pv(g - 1, g - 1 == g_first);
     }
   } else {
-    // =========================== softmax ===========================
-    const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
-    const int row = quarter * 32 + lane;        // query row of this thread
+    // =========================== softmax (two halves) ===========================
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int h = warp >> 2;                   // which Q tile
+    const int quarter = warp & 3;              // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;       // query row of this thread in its tile
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + kTmemS + 128 * h;
+    const uint32_t tO = tmem + lane_addr + kTmemO + 128 * h;
     uint32_t g = 0;
     bool ok = true;
     const float sl2 = p.scale_log2;
@@ -438,110 +508,112 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       const int w = item_index(k);
       if (w >= num_items) break;
       const ItemInfo it = load_item(p, w);
-      const int jq = it.qtile * QT + row;
+      const int head = pair_heads ? it.head0 + h : it.head0;
+      const int qt = pair_heads ? it.qt0 : it.qt0 + h;
+      const int jq = qt * QT + row;
       const bool row_valid = jq < it.ql;
       const int pos = row_valid ? it.L - it.ql + jq : -1;  // last visible key
       const int nblk = (it.L + kBlockSize - 1) / kBlockSize;
       const int shift = nblk * kBlockSize - it.L;
-      const int min_pos = it.L - it.ql + it.qtile * QT;    // smallest position in the tile
+      const int min_pos = it.L - it.ql + qt * QT;          // smallest position in the tile
       float m_run = -INFINITY, l_run = 0.f;
       const uint32_t g_first = g;
       for (int t = 0; t < it.ntiles && ok; ++t, ++g) {
-        ok = wait_bar(bar(kBarSFull0 + (g & 1)), (g >> 1) & 1, abort_flag, status);
+        // S_h of tile g is complete; so is P.V of tile g-1 (issued before it)
+        ok = wait_bar(bar(kBarSFull + h), g & 1, abort_flag, status);
         if (!ok) break;
         tc_fence_after();
         uint32_t sr[KT];
-        {
-          const uint32_t ta = tmem + lane_addr + kTmemS + (g & 1) * KT;
-          tmem_ld32_at<0>(ta, sr);
-          tmem_ld32_at<32>(ta + 32, sr);
-          tmem_ld32_at<64>(ta + 64, sr);
-          tmem_ld32_at<96>(ta + 96, sr);
-        }
+        tmem_ld32_at<0>(tS, sr);
+        tmem_ld32_at<32>(tS + 32, sr);
+        tmem_ld32_at<64>(tS + 64, sr);
+        tmem_ld32_at<96>(tS + 96, sr);
         tmem_ld_wait();
         float s[KT];
 #pragma unroll
         for (int n = 0; n < KT; ++n) s[n] = __uint_as_float(sr[n]);
-        // ---- mask: causal limit, the shifted last block, blocks past the sequence
+        // ---- mask (causal limit, the shifted last block, blocks past the
+        // sequence) and the row max of the raw scores, 8 partial maxima
         const bool need_mask = (t * KT + KT - 1 > min_pos) ||
                                ((t + 1) * kTileBlocks > nblk - 1);
-        float mx = -INFINITY;
+        float mxp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mxp[q] = -INFINITY;
         if (need_mask) {
 #pragma unroll
           for (int n = 0; n < KT; ++n) {
             const int lb = t * kTileBlocks + n / kBlockSize, i = n % kBlockSize;
             const int key = lb * kBlockSize + i - (lb == nblk - 1 ? shift : 0);
             const bool vis = lb < nblk && (lb != nblk - 1 || i >= shift) && key <= pos;
-            s[n] = vis ? s[n] * sl2 : -INFINITY;
-            mx = fmaxf(mx, s[n]);
+            s[n] = vis ? s[n] : -INFINITY;
+            mxp[n & 7] = fmaxf(mxp[n & 7], s[n]);
           }
         } else {
 #pragma unroll
-          for (int n = 0; n < KT; ++n) {
-            s[n] *= sl2;
-            mx = fmaxf(mx, s[n]);
-          }
+          for (int n = 0; n < KT; ++n) mxp[n & 7] = fmaxf(mxp[n & 7], s[n]);
         }
-        // ---- running max: moved only when it grows past the threshold
+        const float mx = sl2 * fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                     fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        // ---- running max (log2 units): moved only when it grows past the threshold
         float alpha = 1.f;
         if (mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx > -INFINITY)) {
           alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - mx);
           m_run = mx;
         }
-        const float base_m = (m_run == -INFINITY) ? 0.f : m_run;
-        float sum = 0.f;
+        const float neg_base = (m_run == -INFINITY) ? 0.f : -m_run;
+        float sump[8];
 #pragma unroll
-        for (int n = 0; n < KT; ++n) {
-          s[n] = ex2(s[n] - base_m);
-          sum += s[n];
+        for (int q = 0; q < 8; ++q) sump[q] = 0.f;
+        // ---- P = exp2(S * scale * log2(e) - max), two bf16 per word, written
+        // over the first half of S in 32-word chunks (this thread has read all
+        // of S already)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pw[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = 64 * c + 2 * j;
+            const float e0 = ex2(fmaf(s[n], sl2, neg_base));  // masked: ex2(-inf) = 0
+            const float e1 = ex2(fmaf(s[n + 1], sl2, neg_base));
+            sump[n & 7] += e0;
+            sump[(n + 1) & 7] += e1;
+            pw[j] = pack_bf16x2(e0, e1);
+          }
+          tmem_st32(tS + 32 * c, pw);
         }
+        const float sum = ((sump[0] + sump[1]) + (sump[2] + sump[3])) +
+                          ((sump[4] + sump[5]) + (sump[6] + sump[7]));
         l_run = l_run * alpha + sum;
-        // ---- P (and O) may be touched once the previous P.V has finished
-        if (g > 0) ok = wait_bar(bar(kBarODone), (g - 1) & 1, abort_flag, status);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < KT / 8; ++c) {  // 16-byte chunks of 8 keys
-          const uint32_t w0 = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
-          const uint32_t w1 = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
-          const uint32_t w2 = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
-          const uint32_t w3 = pack_bf16x2(s[8 * c + 6], s[8 * c + 7]);
-          const uint32_t addr = sP + (c / 8) * LY::kPanelBytes + row * 128 +
-                                (((c % 8) ^ (row % 8)) * 16);
-          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(w0), "r"(w1),
-                       "r"(w2), "r"(w3)
-                       : "memory");
-        }
+        // ---- O carries the old max: rescale it (P.V of tile g-1 is complete)
         if (g != g_first && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
-            tmem_ld32(tmem + lane_addr + kTmemO + c * 32, orr);
+            tmem_ld32(tO + c * 32, orr);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e)
               orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st32(tmem + lane_addr + kTmemO + c * 32, orr);
+            tmem_st32(tO + c * 32, orr);
           }
-          tmem_st_wait();
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kBarPFull));
+        if (lane == 0) mbar_arrive(bar(kBarPFull + h));
       }
       if (!ok || it.ntiles == 0) continue;
       // ---- epilogue: O / l to global memory
-      ok = wait_bar(bar(kBarODone), (g - 1) & 1, abort_flag, status);
+      ok = wait_bar(bar(kBarODone + h), (g - 1) & 1, abort_flag, status);
       if (!ok) break;
       tc_fence_after();
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       __nv_bfloat16* orow =
-          (__nv_bfloat16*)p.out + ((int64_t)(it.q0 + jq) * p.num_q_heads + it.head) * D;
+          (__nv_bfloat16*)p.out + ((int64_t)(it.q0 + jq) * p.num_q_heads + head) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
-        tmem_ld32(tmem + lane_addr + kTmemO + c * 32, orr);
+        tmem_ld32(tO + c * 32, orr);
         tmem_ld_wait();
         if (row_valid) {
 #pragma unroll
@@ -555,13 +627,15 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           }
         }
       }
+      // the next item's first P.V overwrites O: every lane has read it
+      tc_fence_before();
     }
   }
 
   // ---- wind down: every role is done (or gave up); free TMEM
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -571,21 +645,34 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
 
 // One CTA: list the prefill items of every sequence with q_len * group > 16,
 // heaviest (most key tiles) first (a counting sort on the tile count), and
-// store the count in ws_items[0].x.
-__global__ void __launch_bounds__(1024) prefill_plan_kernel(const AttnParams p, int max_tiles) {
+// store the count in ws_items[0].x.  An item pairs two q-heads of one kv-head
+// (pair_heads: the group is even) or two consecutive query tiles of one
+// q-head; its tile count covers the later of its two query tiles.
+__device__ __forceinline__ void prefill_item_range(int L, int ql, int pair_heads, int i,
+                                                   int* last_row_pos) {
+  const int hi_tile = pair_heads ? i : 2 * i + 1;
+  const int last_row = min((hi_tile + 1) * QT, ql) - 1;
+  *last_row_pos = L - ql + last_row;
+}
+
+__global__ void __launch_bounds__(1024)
+prefill_plan_kernel(const AttnParams p, int max_tiles, int pair_heads) {
   extern __shared__ int hist[];  // [max_tiles + 1] counters, then running offsets
   asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int i = threadIdx.x; i <= max_tiles; i += blockDim.x) hist[i] = 0;
   __syncthreads();
+  const int per_tile = pair_heads ? p.num_q_heads / 2 : p.num_q_heads;  // items per (seq, tile)
   // pass 1: histogram of items by tile count
   for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
     const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
     if (ql * p.group <= kDecodeRows || ql > L) continue;
     const int nq = (ql + QT - 1) / QT;
-    for (int i = 0; i < nq; ++i) {
-      const int last = L - ql + min((i + 1) * QT, ql) - 1;
+    const int ni = pair_heads ? nq : (nq + 1) / 2;
+    for (int i = 0; i < ni; ++i) {
+      int last;
+      prefill_item_range(L, ql, pair_heads, i, &last);
       const int nt = min(last / KT + 1, max_tiles);
-      atomicAdd(&hist[nt], p.num_q_heads);
+      atomicAdd(&hist[nt], per_tile);
     }
   }
   __syncthreads();
@@ -604,12 +691,17 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(const AttnParams p, 
     const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
     if (ql * p.group <= kDecodeRows || ql > L) continue;
     const int nq = (ql + QT - 1) / QT;
-    for (int i = nq - 1; i >= 0; --i) {
-      const int last = L - ql + min((i + 1) * QT, ql) - 1;
+    const int ni = pair_heads ? nq : (nq + 1) / 2;
+    for (int i = ni - 1; i >= 0; --i) {
+      int last;
+      prefill_item_range(L, ql, pair_heads, i, &last);
       const int nt = min(last / KT + 1, max_tiles);
-      const int at = atomicAdd(&hist[nt], p.num_q_heads);
-      for (int h = 0; h < p.num_q_heads; ++h)
-        if (at + h < p.max_items) p.ws_items[1 + at + h] = make_int4(s, i, h, nt);
+      const int at = atomicAdd(&hist[nt], per_tile);
+      for (int h = 0; h < per_tile; ++h) {
+        if (at + h >= p.max_items) break;
+        p.ws_items[1 + at + h] = pair_heads ? make_int4(s, i, 2 * h, nt)
+                                            : make_int4(s, 2 * i, h, nt);
+      }
     }
   }
 }
@@ -663,6 +755,8 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
                 (uint64_t)D * 2, (uint64_t)kBlockSize * D * 2, kBlockSize, 1))
     return cudaErrorInvalidValue;
 
+  // two q-heads of one kv-head share every K/V tile when the group is even
+  const int pair_heads = (p.group % 2 == 0) ? 1 : 0;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -683,7 +777,7 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
                                            (int)cfg.dynamicSmemBytes);
       if (e != cudaSuccess) return e;
     }
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_plan_kernel, p, tiles);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_plan_kernel, p, tiles, pair_heads);
     if (e != cudaSuccess) return e;
   }
   const int upper = num_items >= 0 ? num_items
@@ -702,7 +796,7 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv);
+  return cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, pair_heads);
 }
 
 }  // namespace
