@@ -28,6 +28,7 @@ if ROOT not in sys.path:
 
 METRIC = "decode paged-attn KV GB/s (% of HBM peak); mixed-step query tokens/s"
 WORKLOAD = "decode_tinyllama"
+MIXED_WORKLOAD = "mixed_llama3_8b"
 FLUSH_BYTES = 512 << 20
 
 
@@ -52,15 +53,16 @@ def load_peaks() -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    """nvidia-smi clocks and throttle reasons, sampled in the background; only
+    samples taken inside the marked timed windows are reported."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int, period_ms: int = 20):
         self.proc = None
-        self.gpu = gpu_index
+        self.windows = []
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
@@ -70,29 +72,53 @@ class ClockSampler:
         except (OSError, ValueError):
             self.proc = None
 
+    def window(self):
+        """Context manager marking a timed region (host wall clock)."""
+        sampler = self
+
+        class _W:
+            def __enter__(self_w):
+                self_w.t0 = time.time()
+
+            def __exit__(self_w, *exc):
+                sampler.windows.append((self_w.t0, time.time()))
+                return False
+        return _W()
+
     def stop(self) -> dict:
+        import datetime
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.1)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        sm, smax, reasons = [], [], set()
+        sm, smax, reasons, total = [], [], set(), 0
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
+            total += 1
             try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                mhz, mx = float(f[2]), float(f[3])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            if not any(a - 0.02 <= ts <= b + 0.02 for a, b in self.windows):
+                continue
+            sm.append(mhz)
+            smax.append(mx)
+            for n, v in zip(names, f[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples_in_timed_regions": len(sm), "samples_total": total}
+
+
+def _nullctx():
+    import contextlib
+    return contextlib.nullcontext()
 
 
 def dist_setup(n_gpus: int):
@@ -210,6 +236,92 @@ def bench_reference(args) -> None:
 
 # ---------------------------------------------------------------- GPU arm
 
+def timed_steps(ds, stream, flush, steps: int):
+    """K steps, L2 flushed before each (untimed); per-step CUDA events on the
+    launching stream around the whole step and around the attention call.
+    Returns (mean step ms, mean attention ms)."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        ds.write_new_tokens()
+        ev[i][1].record(stream)
+        ds.attention()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / steps
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    return step_ms, attn_ms
+
+
+def prefill_flops(step) -> int:
+    """Flops of the unmasked (query, key) pairs of the prefill-class sequences
+    (q_len * group > 16): 4 * D * Hq per pair (Q.K^T and P.V)."""
+    g = step.num_q_heads // step.num_kv_heads
+    pairs = 0
+    for ql, L in zip(step.query_lens.tolist(), step.seq_lens.tolist()):
+        if ql * g > 16:
+            pairs += ql * (L - ql) + ql * (ql + 1) // 2
+    return 4 * step.head_dim * step.num_q_heads * pairs
+
+
+def bench_mixed(args, dev, stream, flush, world, clocks):
+    """Mixed prefill + decode step (Llama-3-8B attention shape): query tokens/s,
+    plus the prefill chunks alone against the bf16 tensor peak."""
+    import numpy as np
+    import torch
+    from paged_kv_cache_469_b200.inputs import make_step, workload
+    from paged_kv_cache_469_b200.step import DeviceStep
+    step = workload(MIXED_WORKLOAD)
+    ds = DeviceStep(step, device=str(dev))
+    for _ in range(args.warmup):
+        ds.run()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    n = min(args.steps, 100)
+    with clocks.window() if clocks else _nullctx():
+        step_ms, attn_ms = timed_steps(ds, stream, flush, n)
+    barrier(world)
+    step_ms = max_over_ranks(step_ms, world)
+    tokens = sum_over_ranks(step.num_tokens, world)
+    kv_dec = int(sum(L for L, q in zip(step.seq_lens.tolist(), step.query_lens.tolist())
+                     if q * 4 <= 16)) * 2 * step.num_kv_heads * step.head_dim * 2
+    del ds
+    torch.cuda.empty_cache()
+    # the same step's prefill chunks alone (same lengths, same shape)
+    idx = [i for i, q in enumerate(step.query_lens.tolist()) if q * 4 > 16]
+    pre = make_step(name="mixed_prefill_only", dtype="bf16", num_q_heads=step.num_q_heads,
+                    num_kv_heads=step.num_kv_heads, head_dim=step.head_dim,
+                    num_blocks=int(np.sum((step.seq_lens[idx] + 15) // 16)) + 64,
+                    seq_lens=step.seq_lens[idx], query_lens=step.query_lens[idx],
+                    seed=step.seed)
+    dp = DeviceStep(pre, device=str(dev))
+    for _ in range(args.warmup):
+        dp.run()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    with clocks.window() if clocks else _nullctx():
+        _, pre_ms = timed_steps(dp, stream, flush, n)
+    barrier(world)
+    pre_ms = max_over_ranks(pre_ms, world)
+    flops = prefill_flops(pre)
+    peaks = load_peaks()
+    tflops = flops / (pre_ms / 1e3) / 1e12
+    del dp
+    torch.cuda.empty_cache()
+    return {"workload": MIXED_WORKLOAD, "value": round(tokens / (step_ms / 1e3), 1),
+            "unit": "query tokens/s", "ms_per_step": round(step_ms, 4), "steps": n,
+            "query_tokens_per_step_per_gpu": step.num_tokens,
+            "decode_kv_bytes_per_step_per_gpu": kv_dec,
+            "prefill_only": {"ms": round(pre_ms, 4), "gflop": round(flops / 1e9, 3),
+                             "tflops": round(tflops, 1),
+                             "frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
+                             "frac_of_bf16_sustained": round(
+                                 tflops / peaks["bf16_tflops_sustained"], 4),
+                             "peak_source": peaks["source"]}}
+
+
 def bench_ours(args) -> None:
     import numpy as np
     import torch
@@ -230,22 +342,12 @@ def bench_ours(args) -> None:
     for _ in range(args.warmup):
         ds.run()
     torch.cuda.synchronize(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clocks = ClockSampler(local) if rank == 0 or world > 1 else None
     barrier(world)
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.zero_()
-        ev[i][0].record(stream)
-        ds.write_new_tokens()
-        ev[i][1].record(stream)
-        ds.attention()
-        ev[i][2].record(stream)
-    torch.cuda.synchronize(dev)
+    with clocks.window() if clocks else _nullctx():
+        step_ms, attn_ms = timed_steps(ds, stream, flush, args.steps)
     barrier(world)
-    clk = clocks.stop() if clocks else None
-    step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / args.steps
-    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     step_ms_max = max_over_ranks(step_ms, world)
     attn_ms_max = max_over_ranks(attn_ms, world)
     bytes_rank = kv_bytes(step)
@@ -278,15 +380,20 @@ def bench_ours(args) -> None:
     ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.zero_()
-        ev2[i][0].record(stream)
-        e2e_step()
-        ev2[i][1].record(stream)
-    torch.cuda.synchronize(dev)
+    with clocks.window() if clocks else _nullctx():
+        for i in range(args.steps):
+            flush.zero_()
+            ev2[i][0].record(stream)
+            e2e_step()
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / args.steps, world)
     e2e_value = bytes_all / (e2e_ms / 1e3) / 1e9
+    del ds, host_in, dev_view
+    torch.cuda.empty_cache()
+    mixed = None if args.no_mixed else bench_mixed(args, dev, stream, flush, world, clocks)
+    clk = clocks.stop() if clocks else None
 
     if rank != 0:
         if world > 1:
@@ -320,6 +427,7 @@ def bench_ours(args) -> None:
                        "parallelism": f"{world} independent replicas"},
             "attention_ms": round(attn_ms_max, 5),
             "gpu_launches": 2 * args.steps,
+            "mixed_step": mixed,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clk}
@@ -332,10 +440,12 @@ def bench_ours(args) -> None:
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mixed", action="store_true",
+                    help="skip the mixed prefill+decode leg (Llama-3-8B shape)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
