@@ -30,6 +30,10 @@ METRIC = "decode paged-attn KV GB/s (% of HBM peak); mixed-step query tokens/s"
 WORKLOAD = "decode_tinyllama"
 MIXED_WORKLOAD = "mixed_llama3_8b"
 FLUSH_BYTES = 512 << 20
+# dram__bytes_read.sum + dram__bytes_write.sum of one decode_splitk_kernel<64,0,4,4>
+# launch on this workload, from an ncu --set full capture of that launch; set
+# to None whenever that kernel changes, until it is captured again
+DECODE_TRAFFIC_BYTES = 68_939_264 + 1_123_840
 
 
 def kv_bytes(step, seqs=None) -> int:
@@ -271,7 +275,7 @@ def bench_mixed(args, dev, stream, flush, world, clocks):
     plus the prefill chunks alone against the bf16 tensor peak."""
     import numpy as np
     import torch
-    from paged_kv_cache_469_b200.inputs import make_step, workload
+    from paged_kv_cache_469_b200.inputs import prefill_part, workload
     from paged_kv_cache_469_b200.step import DeviceStep
     step = workload(MIXED_WORKLOAD)
     ds = DeviceStep(step, device=str(dev))
@@ -290,12 +294,7 @@ def bench_mixed(args, dev, stream, flush, world, clocks):
     del ds
     torch.cuda.empty_cache()
     # the same step's prefill chunks alone (same lengths, same shape)
-    idx = [i for i, q in enumerate(step.query_lens.tolist()) if q * 4 > 16]
-    pre = make_step(name="mixed_prefill_only", dtype="bf16", num_q_heads=step.num_q_heads,
-                    num_kv_heads=step.num_kv_heads, head_dim=step.head_dim,
-                    num_blocks=int(np.sum((step.seq_lens[idx] + 15) // 16)) + 64,
-                    seq_lens=step.seq_lens[idx], query_lens=step.query_lens[idx],
-                    seed=step.seed)
+    pre = prefill_part(step)
     dp = DeviceStep(pre, device=str(dev))
     for _ in range(args.warmup):
         dp.run()
@@ -405,7 +404,8 @@ def bench_ours(args) -> None:
     achieved = bytes_rank / (attn_ms_max / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "kernel": "decode_splitk_kernel<64,false>",
+                "traffic": DECODE_TRAFFIC_BYTES, "traffic_unit": "bytes per launch (ncu)",
+                "kernel": "decode_splitk_kernel<64,0,4,4>",
                 "peak_source": f"{peaks['source']} HBM copy bandwidth (burst)",
                 "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)}
     cpu = None

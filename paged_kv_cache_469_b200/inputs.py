@@ -209,6 +209,19 @@ def workload(name: str, *, with_values: bool = True) -> StepInputs:
     raise KeyError(name)
 
 
+def prefill_part(step: StepInputs, decode_rows: int = 16) -> StepInputs:
+    """A step of the same shape holding only ``step``'s prefill-class sequences
+    (q_len * group > ``decode_rows``), with the same lengths, fresh draws from
+    the same seed and a pool just large enough for them."""
+    g = step.num_q_heads // step.num_kv_heads
+    idx = [i for i, q in enumerate(step.query_lens.tolist()) if q * g > decode_rows]
+    lens, qls = step.seq_lens[idx], step.query_lens[idx]
+    return make_step(name=f"{step.name}_prefill_only", dtype=step.dtype,
+                     num_q_heads=step.num_q_heads, num_kv_heads=step.num_kv_heads,
+                     head_dim=step.head_dim, num_blocks=int(np.sum((lens + 15) // 16)) + 64,
+                     seq_lens=lens, query_lens=qls, seed=step.seed)
+
+
 def random_step(seed: int, *, dtype: str = "bf16", num_q_heads: int = 8, num_kv_heads: int = 2,
                 head_dim: int = 64, num_seqs: int = 4, max_ctx: int = 100, max_q: int = 20,
                 num_blocks: int | None = None, shared_prefix_tokens: int = 0) -> StepInputs:
