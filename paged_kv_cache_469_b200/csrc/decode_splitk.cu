@@ -400,23 +400,52 @@ decode_splitk_kernel(const AttnParams p) {
   }
   __syncthreads();
   if (!sh_last) return;
-  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
-    const int row = idx / D, d = idx % D;
-    const int64_t base_slot = (int64_t)unit * p.max_parts * kDecodeRows + row;
+  // every partition's (max, sum) per row into shared memory (one round of
+  // loads), then the rows' weights, then one round of 16-byte partial loads
+  // per output chunk (the ring is free: every warp is past its last copy)
+  float* sh_pm = reinterpret_cast<float*>(smem);  // [nparts][kDecodeRows] max, then weight
+  float* sh_pl = sh_pm + nparts * kDecodeRows;    // [nparts][kDecodeRows] sum
+  float* sh_inv = sh_pl + nparts * kDecodeRows;   // [kDecodeRows] 1 / merged sum
+  const int64_t unit_slot = (int64_t)unit * p.max_parts * kDecodeRows;
+  for (int i = threadIdx.x; i < nparts * rows; i += blockDim.x) {
+    const int q = i / rows, row = i % rows;
+    const float2 ml =
+        __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + unit_slot + q * kDecodeRows + row);
+    sh_pm[q * kDecodeRows + row] = ml.x;
+    sh_pl[q * kDecodeRows + row] = ml.y;
+  }
+  __syncthreads();
+  if (threadIdx.x < rows) {
+    const int row = threadIdx.x;
     float M = -INFINITY;
-    for (int q = 0; q < nparts; ++q)
-      M = fmaxf(M, __ldcg(p.ws_ml + (base_slot + (int64_t)q * kDecodeRows) * 2));
+    for (int q = 0; q < nparts; ++q) M = fmaxf(M, sh_pm[q * kDecodeRows + row]);
     const float base = (M == -INFINITY) ? 0.f : M;
-    float Ls = 0.f, Os = 0.f;
+    float Ls = 0.f;
     for (int q = 0; q < nparts; ++q) {
-      const int64_t slot = base_slot + (int64_t)q * kDecodeRows;
-      const float f = exp2f(__ldcg(p.ws_ml + slot * 2) - base);
-      Ls += __ldcg(p.ws_ml + slot * 2 + 1) * f;
-      Os += __ldcg(p.ws_o + slot * D + d) * f;
+      const float f = exp2f(sh_pm[q * kDecodeRows + row] - base);
+      sh_pm[q * kDecodeRows + row] = f;
+      Ls += sh_pl[q * kDecodeRows + row] * f;
     }
+    sh_inv[row] = Ls > 0.f ? 1.f / Ls : 0.f;
+  }
+  __syncthreads();
+  constexpr int D4 = D / 4;
+  const float4* po = reinterpret_cast<const float4*>(p.ws_o);
+  for (int i = threadIdx.x; i < rows * D4; i += blockDim.x) {
+    const int row = i / D4, d4 = i % D4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int q = 0; q < nparts; ++q) {
+      const float4 v = __ldcg(po + (unit_slot + q * kDecodeRows + row) * D4 + d4);
+      const float f = sh_pm[q * kDecodeRows + row];
+      acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+    }
+    const float inv = sh_inv[row];
     const int tok = q0 + row / G, head = kvh * G + row % G;
-    out[((int64_t)tok * p.num_q_heads + head) * D + d] =
-        __float2bfloat16_rn(Ls > 0.f ? Os / Ls : 0.f);
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(out + ((int64_t)tok * p.num_q_heads + head) * D + 4 * d4) = pk;
   }
   if (threadIdx.x == 0) p.ws_counter[unit] = 0;  // ready for the next call
 }
@@ -427,7 +456,10 @@ cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
   auto kernel = decode_splitk_kernel<D, kRows16, kStages, kWarps>;
   const int ring = kWarps * kStages * DecodeSmem<D>::kSlotBytes;
   const int merge = kWarps * kDecodeRows * D * (int)sizeof(float);
-  const int smem = ring > merge ? ring : merge;
+  // the cross-partition merge: (max, sum) per partition and row, 1 / sum per row
+  const int split = (2 * p.max_parts + 1) * kDecodeRows * (int)sizeof(float);
+  int smem = ring > merge ? ring : merge;
+  if (split > smem) smem = split;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

@@ -167,6 +167,7 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
 
   const WorkspaceLayout w =
       workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len);
+  if (w.max_parts > kDecodeMaxParts) return PA_ERR_UNSUPPORTED;
   AttnParams p{};
   p.out = out;
   p.q = q;

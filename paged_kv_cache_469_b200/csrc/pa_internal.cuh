@@ -10,6 +10,10 @@ namespace pa {
 
 constexpr int kBlockSize = 16;       // tokens per cache block (the pages' default)
 constexpr int kDecodeRows = 16;      // query rows per kv-head one decode CTA holds (MMA M)
+// split-K partitions per sequence the decode kernel can merge (its shared
+// memory holds each partition's per-row max and sum): 1536 partitions of at
+// least 1024 keys, i.e. sequences of at least 1.5M tokens
+constexpr int kDecodeMaxParts = 1536;
 #ifndef PA_DECODE_WARPS
 #define PA_DECODE_WARPS 4
 #endif

@@ -36,6 +36,7 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include "pa_fastmath.cuh"
 #include "pa_internal.cuh"
 
 namespace pa {
@@ -61,7 +62,18 @@ constexpr uint32_t kTmemCols = 512;
 // two per column) written over the first 64 columns of S once S is read
 constexpr uint32_t kTmemO = 0, kTmemS = 256;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
+// longest single sleep of a waiting thread before it checks the limit again
+#ifndef PA_WAIT_SUSPEND_NS
+#define PA_WAIT_SUSPEND_NS 20000
+#endif
+constexpr uint32_t kWaitSuspendNs = PA_WAIT_SUSPEND_NS;
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: move the max only past 2^8
+// of every 8 pairs of score columns, how many take exp2 on the FMA pipe
+// (exp2_poly2) instead of the exponential unit
+#ifndef PA_PREFILL_POLY_PAIRS
+#define PA_PREFILL_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = PA_PREFILL_POLY_PAIRS;
 
 template <int D>
 struct PrefillLayout {
@@ -121,6 +133,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same, but a thread whose phase has not completed sleeps until it does,
+// or for at most suspend_ns, instead of returning at once: waiting warps then
+// take no issue slots from the warps that share their scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
 
 // Wait for the phase of `bar` with parity `parity` to complete.  Gives up
 // (returns false) when another role of the CTA has given up, or after the time
@@ -130,7 +156,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSuspendNs)) return true;
     if (*abort_flag) return false;
     if (globaltimer() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -246,11 +272,6 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -532,28 +553,31 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         float s[KT];
 #pragma unroll
         for (int n = 0; n < KT; ++n) s[n] = __uint_as_float(sr[n]);
-        // ---- mask (causal limit, the shifted last block, blocks past the
-        // sequence) and the row max of the raw scores, 8 partial maxima
-        const bool need_mask = (t * KT + KT - 1 > min_pos) ||
-                               ((t + 1) * kTileBlocks > nblk - 1);
-        float mxp[8];
+        // ---- mask: column 16 b + i holds key t*KT + 16 b + i for blocks before
+        // the sequence's last block; the last block was loaded shifted down by
+        // `shift` rows, so its column 16 b + i holds key t*KT + 16 b + i - shift
+        // and its first `shift` columns are empty; columns past it are empty.
+        // Per block, slots lo .. hi are visible to this row.
+        if (t * KT + KT - 1 > min_pos || (t + 1) * kTileBlocks > nblk - 1) {
+          const int lim = pos - t * KT;  // last visible key, tile-relative
+          const int lastb = nblk - 1 - t * kTileBlocks;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) mxp[q] = -INFINITY;
-        if (need_mask) {
+          for (int b = 0; b < kTileBlocks; ++b) {
+            const int lo = b < lastb ? 0 : (b == lastb ? shift : 16);
+            const int hi = lim - 16 * b + (b == lastb ? shift : 0);
 #pragma unroll
-          for (int n = 0; n < KT; ++n) {
-            const int lb = t * kTileBlocks + n / kBlockSize, i = n % kBlockSize;
-            const int key = lb * kBlockSize + i - (lb == nblk - 1 ? shift : 0);
-            const bool vis = lb < nblk && (lb != nblk - 1 || i >= shift) && key <= pos;
-            s[n] = vis ? s[n] : -INFINITY;
-            mxp[n & 7] = fmaxf(mxp[n & 7], s[n]);
+            for (int i = 0; i < 16; ++i)
+              s[16 * b + i] = (i >= lo && i <= hi) ? s[16 * b + i] : -INFINITY;
           }
-        } else {
-#pragma unroll
-          for (int n = 0; n < KT; ++n) mxp[n & 7] = fmaxf(mxp[n & 7], s[n]);
         }
-        const float mx = sl2 * fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                                     fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        // ---- row max of the raw scores: four chains of three-input maxima
+        float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int n = 0; n < KT; n += 8) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mc[q] = max3(mc[q], s[n + 2 * q], s[n + 2 * q + 1]);
+        }
+        const float mx = sl2 * max3(mc[0], mc[1], fmaxf(mc[2], mc[3]));
         // ---- running max (log2 units): moved only when it grows past the threshold
         float alpha = 1.f;
         if (mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx > -INFINITY)) {
@@ -561,39 +585,56 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           m_run = mx;
         }
         const float neg_base = (m_run == -INFINITY) ? 0.f : -m_run;
-        float sump[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) sump[q] = 0.f;
-        // ---- P = exp2(S * scale * log2(e) - max), two bf16 per word, written
-        // over the first half of S in 32-word chunks (this thread has read all
-        // of S already)
+        // ---- P = exp2(S * scale * log2(e) - max) on pairs of columns: kPolyPairs
+        // of every 8 pairs on the FMA pipe, the rest on the exponential unit;
+        // two bf16 per word, written over the first half of S in 32-word
+        // chunks (this thread has read all of S already)
+        const uint64_t scale2 = f2(sl2, sl2), base2 = f2(neg_base, neg_base);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pw[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int n = 64 * c + 2 * j;
-            const float e0 = ex2(fmaf(s[n], sl2, neg_base));  // masked: ex2(-inf) = 0
-            const float e1 = ex2(fmaf(s[n + 1], sl2, neg_base));
-            sump[n & 7] += e0;
-            sump[(n + 1) & 7] += e1;
+            const uint64_t x = fma2(f2(s[n], s[n + 1]), scale2, base2);
+            uint64_t e;
+            if ((j & 7) < kPolyPairs) {
+              e = exp2_poly2(x);
+            } else {
+              float x0, x1;
+              f2_split(x, x0, x1);
+              e = f2(ex2(x0), ex2(x1));  // masked: ex2(-inf) = 0
+            }
+            acc[j & 3] = add2(acc[j & 3], e);
+            float e0, e1;
+            f2_split(e, e0, e1);
             pw[j] = pack_bf16x2(e0, e1);
           }
           tmem_st32(tS + 32 * c, pw);
         }
-        const float sum = ((sump[0] + sump[1]) + (sump[2] + sump[3])) +
-                          ((sump[4] + sump[5]) + (sump[6] + sump[7]));
+        float sum;
+        {
+          float a0, a1;
+          f2_split(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), a0, a1);
+          sum = a0 + a1;
+        }
         l_run = l_run * alpha + sum;
         // ---- O carries the old max: rescale it (P.V of tile g-1 is complete)
         if (g != g_first && __any_sync(0xffffffffu, alpha != 1.f)) {
+          const uint64_t alpha2 = f2(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
             tmem_ld32(tO + c * 32, orr);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            for (int e = 0; e < 16; ++e) {
+              uint32_t lo, hi;
+              u2_split(mul2(u2(orr[2 * e], orr[2 * e + 1]), alpha2), lo, hi);
+              orr[2 * e] = lo;
+              orr[2 * e + 1] = hi;
+            }
             tmem_st32(tO + c * 32, orr);
           }
         }
