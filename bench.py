@@ -7,10 +7,15 @@ pool), bf16, synthetic N(0,1) data.
 
 Prints ONE JSON line (rank 0).  `value` is decode KV GB/s: the K/V bytes the
 step's attention must read (sum over sequences of seq_len * 2 * Hkv * D * 2 B,
-summed over ranks) divided by the device time of a step (max over ranks).  L2
-is flushed (a 512 MiB write) before every timed step and the flush is not
-timed.  `--impl reference` times the CPU oracle on a bounded sample of the same
-workload instead.
+summed over ranks) divided by the device time of a step (max over ranks).
+Steps run back to back, as in a serving loop, each one a replay of a CUDA
+graph of the step's launches (the plain stream launches are timed too and
+reported beside it).  No step finds its inputs in L2:
+when one step reads less than twice the L2 size, the timed loop rotates over
+that many identical copies of the workload (own pool, own tensors) that
+consecutive reads of one copy are separated by more than twice the L2 size of
+other traffic.  `--impl reference` times the CPU oracle on a bounded sample of
+the same workload instead.
 """
 from __future__ import annotations
 
@@ -29,11 +34,12 @@ if ROOT not in sys.path:
 METRIC = "decode paged-attn KV GB/s (% of HBM peak); mixed-step query tokens/s"
 WORKLOAD = "decode_tinyllama"
 MIXED_WORKLOAD = "mixed_llama3_8b"
-FLUSH_BYTES = 512 << 20
+L2_BYTES = 126 * 1000 * 1000  # B200 L2, for sizing the rotation of workload copies
+MAX_COPIES = 8
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode_splitk_kernel<64,0,4,4>
 # launch on this workload, from an ncu --set full capture of that launch; set
 # to None whenever that kernel changes, until it is captured again
-DECODE_TRAFFIC_BYTES = 68_939_264 + 1_123_840
+DECODE_TRAFFIC_BYTES = None
 
 
 def kv_bytes(step, seqs=None) -> int:
@@ -240,23 +246,32 @@ def bench_reference(args) -> None:
 
 # ---------------------------------------------------------------- GPU arm
 
-def timed_steps(ds, stream, flush, steps: int):
-    """K steps, L2 flushed before each (untimed); per-step CUDA events on the
-    launching stream around the whole step and around the attention call.
-    Returns (mean step ms, mean attention ms)."""
+def step_bytes(step) -> int:
+    """Bytes one step touches in HBM at least: the K/V it reads plus q and out."""
+    elem = 4 if step.dtype == "f32" else 2
+    return kv_bytes(step) + 2 * int(step.q.size) * elem
+
+
+def copies_for(step) -> int:
+    """Copies of the workload to rotate over so that no step finds its inputs in
+    L2: enough that the other copies' traffic between two reads of one copy
+    exceeds twice the L2 size."""
+    b = max(1, step_bytes(step))
+    return int(min(MAX_COPIES, max(1, -(-2 * L2_BYTES // b) + 1))) if b < 2 * L2_BYTES else 1
+
+
+def timed_loop(fns, stream, steps: int) -> float:
+    """Mean device ms per call over `steps` back-to-back calls of fns[i % len(fns)]
+    (CUDA events on the launching stream around the whole loop)."""
     import torch
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
     for i in range(steps):
-        flush.zero_()
-        ev[i][0].record(stream)
-        ds.write_new_tokens()
-        ev[i][1].record(stream)
-        ds.attention()
-        ev[i][2].record(stream)
+        fns[i % len(fns)]()
+    b.record(stream)
     torch.cuda.synchronize()
-    step_ms = sum(e[0].elapsed_time(e[2]) for e in ev) / steps
-    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
-    return step_ms, attn_ms
+    return a.elapsed_time(b) / steps
 
 
 def prefill_flops(step) -> int:
@@ -270,55 +285,60 @@ def prefill_flops(step) -> int:
     return 4 * step.head_dim * step.num_q_heads * pairs
 
 
-def bench_mixed(args, dev, stream, flush, world, clocks):
+def bench_mixed(args, dev, stream, world, clocks):
     """Mixed prefill + decode step (Llama-3-8B attention shape): query tokens/s,
     plus the prefill chunks alone against the bf16 tensor peak."""
-    import numpy as np
     import torch
     from paged_kv_cache_469_b200.inputs import prefill_part, workload
     from paged_kv_cache_469_b200.step import DeviceStep
     step = workload(MIXED_WORKLOAD)
-    ds = DeviceStep(step, device=str(dev))
-    for _ in range(args.warmup):
-        ds.run()
+    n = min(args.steps, 200)
+    dss = [DeviceStep(step, device=str(dev)) for _ in range(copies_for(step))]
+    graphs = [d.capture("step") for d in dss]
+    for i in range(args.warmup):
+        graphs[i % len(dss)].replay()
     torch.cuda.synchronize(dev)
     barrier(world)
-    n = min(args.steps, 100)
     with clocks.window() if clocks else _nullctx():
-        step_ms, attn_ms = timed_steps(ds, stream, flush, n)
+        step_ms = timed_loop([g.replay for g in graphs], stream, n)
     barrier(world)
     step_ms = max_over_ranks(step_ms, world)
     tokens = sum_over_ranks(step.num_tokens, world)
+    g = step.num_q_heads // step.num_kv_heads
     kv_dec = int(sum(L for L, q in zip(step.seq_lens.tolist(), step.query_lens.tolist())
-                     if q * 4 <= 16)) * 2 * step.num_kv_heads * step.head_dim * 2
-    del ds
+                     if q * g <= 16)) * 2 * step.num_kv_heads * step.head_dim * 2
+    copies = len(dss)
+    del dss, graphs
     torch.cuda.empty_cache()
     # the same step's prefill chunks alone (same lengths, same shape)
     pre = prefill_part(step)
-    dp = DeviceStep(pre, device=str(dev))
-    for _ in range(args.warmup):
-        dp.run()
+    dps = [DeviceStep(pre, device=str(dev)) for _ in range(copies_for(pre))]
+    pgraphs = [d.capture("attention") for d in dps]
+    for i in range(args.warmup):
+        pgraphs[i % len(dps)].replay()
     torch.cuda.synchronize(dev)
     barrier(world)
     with clocks.window() if clocks else _nullctx():
-        _, pre_ms = timed_steps(dp, stream, flush, n)
+        pre_ms = timed_loop([g.replay for g in pgraphs], stream, n)
     barrier(world)
     pre_ms = max_over_ranks(pre_ms, world)
     flops = prefill_flops(pre)
     peaks = load_peaks()
     tflops = flops / (pre_ms / 1e3) / 1e12
-    del dp
+    pre_copies = len(dps)
+    del dps, pgraphs
     torch.cuda.empty_cache()
     return {"workload": MIXED_WORKLOAD, "value": round(tokens / (step_ms / 1e3), 1),
             "unit": "query tokens/s", "ms_per_step": round(step_ms, 4), "steps": n,
             "query_tokens_per_step_per_gpu": step.num_tokens,
-            "decode_kv_bytes_per_step_per_gpu": kv_dec,
+            "decode_kv_bytes_per_step_per_gpu": kv_dec, "copies_rotated": copies,
             "prefill_only": {"ms": round(pre_ms, 4), "gflop": round(flops / 1e9, 3),
                              "tflops": round(tflops, 1),
                              "frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
                              "frac_of_bf16_sustained": round(
                                  tflops / peaks["bf16_tflops_sustained"], 4),
-                             "peak_source": peaks["source"]}}
+                             "peak_source": peaks["source"], "copies_rotated": pre_copies,
+                             "kernels": "prefill_plan_kernel + prefill_tcgen05_kernel<128>"}}
 
 
 def bench_ours(args) -> None:
@@ -333,65 +353,96 @@ def bench_ours(args) -> None:
     dev = torch.device("cuda", local if world > 1 else 0)
     lib.library()
     step = workload(WORKLOAD)
-    ds = DeviceStep(step, device=str(dev))
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    dss = [DeviceStep(step, device=str(dev)) for _ in range(copies_for(step))]
+    copies = len(dss)
 
-    # ---- device-resident step: warm-up, then K timed steps (L2 flushed before each)
-    for _ in range(args.warmup):
-        ds.run()
+    # ---- device-resident steps, back to back over the rotating copies: one
+    # CUDA graph replay per step (and, for reference, plain stream launches)
+    step_graphs = [d.capture("step") for d in dss]
+    attn_graphs = [d.capture("attention") for d in dss]
+    for i in range(args.warmup):
+        step_graphs[i % copies].replay()
+        dss[i % copies].run()
     torch.cuda.synchronize(dev)
     clocks = ClockSampler(local) if rank == 0 or world > 1 else None
     barrier(world)
     torch.cuda.synchronize(dev)
     with clocks.window() if clocks else _nullctx():
-        step_ms, attn_ms = timed_steps(ds, stream, flush, args.steps)
+        step_ms = timed_loop([g.replay for g in step_graphs], stream, args.steps)
     barrier(world)
+    torch.cuda.synchronize(dev)
+    # the attention call alone (the roofline's kernel): back-to-back stream
+    # launches, each a programmatic dependent of the one before, so that the
+    # interval is the kernel's own time (a one-kernel graph per call would add
+    # its launch gap)
+    with clocks.window() if clocks else _nullctx():
+        attn_ms = timed_loop([d.attention for d in dss], stream, args.steps)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with clocks.window() if clocks else _nullctx():
+        attn_graph_ms = timed_loop([g.replay for g in attn_graphs], stream, args.steps)
+    barrier(world)
+    attn_graph_ms = max_over_ranks(attn_graph_ms, world)
+    torch.cuda.synchronize(dev)
+    with clocks.window() if clocks else _nullctx():
+        stream_step_ms = timed_loop([d.run for d in dss], stream, args.steps)
+    barrier(world)
+    stream_step_ms = max_over_ranks(stream_step_ms, world)
     step_ms_max = max_over_ranks(step_ms, world)
     attn_ms_max = max_over_ranks(attn_ms, world)
     bytes_rank = kv_bytes(step)
     bytes_all = sum_over_ranks(bytes_rank, world)
     value = bytes_all / (step_ms_max / 1e3) / 1e9
 
-    # ---- end to end through the public API from pinned host buffers
+    # ---- end to end through the public API from pinned host buffers: every step
+    # copies its inputs in, runs, and copies its output back
+    ds0 = dss[0]
     host_in = {k: torch.from_numpy(np.ascontiguousarray(a)) for k, a in (
         ("q", step.q), ("k_new", step.k_new), ("v_new", step.v_new),
-        ("slot_mapping", ds.plan.slot_mapping), ("block_tables", ds.plan.block_tables),
-        ("seq_lens", ds.plan.seq_lens), ("query_start_loc", ds.plan.query_start_loc))}
+        ("slot_mapping", ds0.plan.slot_mapping), ("block_tables", ds0.plan.block_tables),
+        ("seq_lens", ds0.plan.seq_lens), ("query_start_loc", ds0.plan.query_start_loc))}
     host_in = {k: v.pin_memory() for k, v in host_in.items()}
-    host_out = torch.empty(ds.out.shape, dtype=torch.int16).pin_memory()
-    dev_view = {"q": ds.q.view(torch.int16), "k_new": ds.k_new.view(torch.int16),
-                "v_new": ds.v_new.view(torch.int16), "slot_mapping": ds.slot_mapping,
-                "block_tables": ds.block_tables, "seq_lens": ds.seq_lens,
-                "query_start_loc": ds.query_start_loc}
+    host_out = torch.empty(ds0.out.shape, dtype=torch.int16).pin_memory()
+    dev_views = [{"q": d.q.view(torch.int16), "k_new": d.k_new.view(torch.int16),
+                  "v_new": d.v_new.view(torch.int16), "slot_mapping": d.slot_mapping,
+                  "block_tables": d.block_tables, "seq_lens": d.seq_lens,
+                  "query_start_loc": d.query_start_loc} for d in dss]
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = host_out.numel() * host_out.element_size()
 
-    def e2e_step():
+    def e2e_step(i):
+        d, view = dss[i % copies], dev_views[i % copies]
         for k, hv in host_in.items():
-            dev_view[k].copy_(hv.view(dev_view[k].dtype), non_blocking=True)
-        ds.run()
-        host_out.copy_(ds.out.view(torch.int16), non_blocking=True)
+            view[k].copy_(hv.view(view[k].dtype), non_blocking=True)
+        d.run()
+        host_out.copy_(d.out.view(torch.int16), non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    def e2e_graph(r):
+        d, view = dss[r], dev_views[r]
+
+        def copies_in():
+            for k, hv in host_in.items():
+                view[k].copy_(hv.view(view[k].dtype), non_blocking=True)
+
+        def copy_out():
+            host_out.copy_(d.out.view(torch.int16), non_blocking=True)
+        return d.capture("step", prologue=copies_in, epilogue=copy_out)
+
+    e2e_graphs = [e2e_graph(r) for r in range(copies)]
+    for i in range(args.warmup):
+        e2e_graphs[i % copies].replay()
     torch.cuda.synchronize(dev)
-    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
     with clocks.window() if clocks else _nullctx():
-        for i in range(args.steps):
-            flush.zero_()
-            ev2[i][0].record(stream)
-            e2e_step()
-            ev2[i][1].record(stream)
-        torch.cuda.synchronize(dev)
+        e2e_ms = timed_loop([g.replay for g in e2e_graphs], stream, args.steps)
     barrier(world)
-    e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev2) / args.steps, world)
+    e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_value = bytes_all / (e2e_ms / 1e3) / 1e9
-    del ds, host_in, dev_view
+    del dss, host_in, dev_views, ds0, step_graphs, attn_graphs, e2e_graphs
     torch.cuda.empty_cache()
-    mixed = None if args.no_mixed else bench_mixed(args, dev, stream, flush, world, clocks)
+    mixed = None if args.no_mixed else bench_mixed(args, dev, stream, world, clocks)
     clk = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -423,9 +474,14 @@ def bench_ours(args) -> None:
                        "context": "U[128,2048]", "num_q_heads": 32, "num_kv_heads": 4,
                        "head_dim": 64, "block_size": 16, "num_blocks": step.num_blocks,
                        "kv_bytes_per_step_per_gpu": bytes_rank,
-                       "l2": "flushed (512 MiB write) before every timed step",
+                       "l2": f"not flushed: inputs larger than L2 (steps rotate over {copies} "
+                             f"copies of the workload, {copies * step_bytes(step) / 1e6:.0f} MB "
+                             f"touched per rotation)",
                        "parallelism": f"{world} independent replicas"},
             "attention_ms": round(attn_ms_max, 5),
+            "launch": "one CUDA graph replay per step (cache write + attention)",
+            "stream_launch_ms_per_step": round(stream_step_ms, 5),
+            "attention_graph_replay_ms": round(attn_graph_ms, 5),
             "gpu_launches": 2 * args.steps,
             "mixed_step": mixed,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),

@@ -133,8 +133,10 @@ decode_splitk_kernel(const AttnParams p) {
 
   // Launched as a programmatic dependent: the CTA may be resident before the
   // preceding kernel on the stream (typically the cache write) has finished;
-  // nothing that kernel may write is read before this wait.
+  // nothing that kernel may write is read before this wait.  The next kernel
+  // may then be launched at once: it waits for this grid in the same way.
   grid_dependency_wait();
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   const int q0 = p.query_start_loc[s];
   const int ql = p.query_start_loc[s + 1] - q0;
@@ -460,7 +462,8 @@ cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
   const int split = (2 * p.max_parts + 1) * kDecodeRows * (int)sizeof(float);
   int smem = ring > merge ? ring : merge;
   if (split > smem) smem = split;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<int> smem_done[64];
+  cudaError_t e = raise_smem_limit(kernel, smem, smem_done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.max_parts, p.num_kv_heads, p.num_seqs);

@@ -6,7 +6,29 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace pa {
+
+// Raise a kernel's dynamic shared-memory limit only when a launch needs more
+// than every earlier launch of it on this device (the attribute persists), so
+// that a steady stream of calls makes no attribute call at all.  `done` is
+// the kernel's own per-device record.
+template <typename Kernel>
+inline cudaError_t raise_smem_limit(Kernel kernel, int bytes, std::atomic<int> (&done)[64]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (done[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) {
+    int cur = done[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !done[dev].compare_exchange_weak(cur, bytes)) {
+    }
+  }
+  return e;
+}
 
 constexpr int kBlockSize = 16;       // tokens per cache block (the pages' default)
 constexpr int kDecodeRows = 16;      // query rows per kv-head one decode CTA holds (MMA M)

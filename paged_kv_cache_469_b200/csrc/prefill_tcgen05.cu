@@ -45,7 +45,12 @@ namespace {
 constexpr int QT = kPrefillQTile;               // 128 query rows per Q tile
 constexpr int KT = kPrefillKvTile;              // 128 keys per K/V tile
 constexpr int kTileBlocks = KT / kBlockSize;    // 8 cache blocks per tile
-constexpr int kKStages = 2, kVStages = 2;
+// K / V tile stages: a K tile is needed one MMA round after V's (P.V of a
+// tile follows its Q K^T), so K benefits first from a deeper ring
+#ifndef PA_PREFILL_K_STAGES
+#define PA_PREFILL_K_STAGES 2
+#endif
+constexpr int kKStages = PA_PREFILL_K_STAGES, kVStages = 2;
 constexpr int kThreads = 384;                   // 12 warps = 3 warpgroups
 // warpgroup 0 (warps 0..3): softmax of half 0; warpgroup 1 (4..7): softmax of
 // half 1 (a warp reads the TMEM lanes 32 * (warp % 4) ..); warpgroup 2: warp
@@ -74,6 +79,12 @@ constexpr float kRescaleThreshold = 8.0f;       // log2 units: move the max only
 #define PA_PREFILL_POLY_PAIRS 0
 #endif
 constexpr int kPolyPairs = PA_PREFILL_POLY_PAIRS;
+// independent max chains over a row of scores (a power of two, at most 32)
+#ifndef PA_PREFILL_MAX_CHAINS
+#define PA_PREFILL_MAX_CHAINS 8
+#endif
+constexpr int kMaxChains = PA_PREFILL_MAX_CHAINS;
+static_assert((kMaxChains & (kMaxChains - 1)) == 0 && kMaxChains <= 32, "max chains");
 
 template <int D>
 struct PrefillLayout {
@@ -90,6 +101,7 @@ struct PrefillLayout {
   // D = 64 would fit two CTAs per SM, whose TMEM allocations would then queue
   // behind each other: ask for enough shared memory to keep one CTA per SM.
   static constexpr int total = (used < 120 * 1024 ? 120 * 1024 : used) + 1024;
+  static_assert(total <= 227 * 1024, "shared memory of one CTA");
 };
 
 // mbarrier indices
@@ -362,8 +374,11 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   tc_fence_after();
   const uint32_t tmem = sh_tmem_base;
 
-  // the work list and the cache must be complete before anything reads them
+  // the work list and the cache must be complete before anything reads them;
+  // the next kernel on the stream may be launched from then on (it waits for
+  // this grid before it reads anything)
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int num_items = p.ws_items[0].x;
   int* status = p.ws_status;
 
@@ -570,14 +585,22 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
               s[16 * b + i] = (i >= lo && i <= hi) ? s[16 * b + i] : -INFINITY;
           }
         }
-        // ---- row max of the raw scores: four chains of three-input maxima
-        float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // ---- row max of the raw scores: kMaxChains independent chains of
+        // three-input maxima, then a tree
+        float mc[kMaxChains];
 #pragma unroll
-        for (int n = 0; n < KT; n += 8) {
+        for (int q = 0; q < kMaxChains; ++q) mc[q] = fmaxf(s[2 * q], s[2 * q + 1]);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) mc[q] = max3(mc[q], s[n + 2 * q], s[n + 2 * q + 1]);
+        for (int n = 2 * kMaxChains; n < KT; n += 2 * kMaxChains) {
+#pragma unroll
+          for (int q = 0; q < kMaxChains; ++q) mc[q] = max3(mc[q], s[n + 2 * q], s[n + 2 * q + 1]);
         }
-        const float mx = sl2 * max3(mc[0], mc[1], fmaxf(mc[2], mc[3]));
+#pragma unroll
+        for (int w = kMaxChains; w > 1; w /= 2) {
+#pragma unroll
+          for (int q = 0; q < w / 2; ++q) mc[q] = fmaxf(mc[q], mc[q + w / 2]);
+        }
+        const float mx = sl2 * mc[0];
         // ---- running max (log2 units): moved only when it grows past the threshold
         float alpha = 1.f;
         if (mx > m_run + kRescaleThreshold || (m_run == -INFINITY && mx > -INFINITY)) {
@@ -699,6 +722,9 @@ __device__ __forceinline__ void prefill_item_range(int L, int ql, int pair_heads
 __global__ void __launch_bounds__(1024)
 prefill_plan_kernel(const AttnParams p, int max_tiles, int pair_heads) {
   extern __shared__ int hist[];  // [max_tiles + 1] counters, then running offsets
+  // the prefill kernel may be launched at once: it waits for this grid before
+  // it reads the work list
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int i = threadIdx.x; i <= max_tiles; i += blockDim.x) hist[i] = 0;
   __syncthreads();
@@ -813,9 +839,9 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cfg.dynamicSmemBytes > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(prefill_plan_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)cfg.dynamicSmemBytes);
+      static std::atomic<int> plan_smem_done[64];
+      cudaError_t e = raise_smem_limit(prefill_plan_kernel, (int)cfg.dynamicSmemBytes,
+                                       plan_smem_done);
       if (e != cudaSuccess) return e;
     }
     cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_plan_kernel, p, tiles, pair_heads);
@@ -828,7 +854,8 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
   const int grid = max(1, min(sm_count(), upper));
   auto kernel = prefill_tcgen05_kernel<D>;
   const int smem = PrefillLayout<D>::total;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<int> smem_done[64];
+  cudaError_t e = raise_smem_limit(kernel, smem, smem_done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

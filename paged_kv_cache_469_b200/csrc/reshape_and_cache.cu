@@ -16,9 +16,12 @@ reshape_and_cache_kernel(const uint4* __restrict__ k, const uint4* __restrict__ 
                          uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                          const int64_t* __restrict__ slot_mapping, int num_tokens,
                          int num_kv_heads, int64_t num_slots) {
-  // let a programmatic dependent (the attention kernel) get launched now; it
-  // waits for this grid's completion before reading the cache
+  // let the next kernel (the attention kernel) get launched now: it waits for
+  // this grid's completion before it reads anything
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  // launched as a programmatic dependent of the previous kernel on the stream:
+  // nothing is read or written before that kernel has completed
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= (int64_t)num_tokens * num_kv_heads) return;
@@ -49,17 +52,27 @@ cudaError_t launch_reshape_and_cache(const void* k, const void* v, void* k_cache
   const int64_t grid = (rows + warps_per_cta - 1) / warps_per_cta;
   const int vec = head_dim * elem_bytes / 16;
   const int64_t num_slots = (int64_t)num_blocks * kBlockSize;
-  auto args = [&](auto kernel) {
-    kernel<<<(unsigned)grid, warps_per_cta * 32, 0, stream>>>(
-        (const uint4*)k, (const uint4*)v, (uint4*)k_cache, (uint4*)v_cache, slot_mapping,
-        num_tokens, num_kv_heads, num_slots);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(warps_per_cta * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto launch = [&](auto kernel) {
+    return cudaLaunchKernelEx(&cfg, kernel, (const uint4*)k, (const uint4*)v, (uint4*)k_cache,
+                              (uint4*)v_cache, slot_mapping, num_tokens, num_kv_heads, num_slots);
   };
+  cudaError_t e;
   switch (vec) {
-    case 8: args(reshape_and_cache_kernel<8>); break;    // bf16 D=64
-    case 16: args(reshape_and_cache_kernel<16>); break;  // bf16 D=128, f32 D=64
-    case 32: args(reshape_and_cache_kernel<32>); break;  // f32 D=128
+    case 8: e = launch(reshape_and_cache_kernel<8>); break;    // bf16 D=64
+    case 16: e = launch(reshape_and_cache_kernel<16>); break;  // bf16 D=128, f32 D=64
+    case 32: e = launch(reshape_and_cache_kernel<32>); break;  // f32 D=128
     default: return cudaErrorInvalidValue;
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -5,7 +5,9 @@ the host (block allocation, slot mapping, super-sequence offsets), puts the
 cache and the step's tensors in device memory, writes the earlier tokens' K/V
 into the cache with ``pa_reshape_and_cache``, and then runs the step itself:
 ``pa_reshape_and_cache`` for the new tokens followed by
-``pa_attention_varlen``.
+``pa_attention_varlen``.  ``capture`` records those launches in a CUDA graph,
+the way a serving loop replays a steady decode step without paying the host
+cost of each call again.
 """
 from __future__ import annotations
 
@@ -78,6 +80,33 @@ class DeviceStep:
         """One step: cache write of the new tokens, then attention."""
         self.write_new_tokens(stream)
         return self.attention(stream, host_hints)
+
+    def capture(self, what: str = "step", prologue=None, epilogue=None) -> torch.cuda.CUDAGraph:
+        """A CUDA graph of this step's launches: "step" (cache write of the new
+        tokens, then attention) or "attention" (the attention call alone).
+        ``prologue`` / ``epilogue`` are captured before / after them (for
+        example host-device copies).  Replaying the graph repeats the step on
+        whatever the step's device tensors hold at that time."""
+        fn = self.run if what == "step" else self.attention
+
+        def body():
+            if prologue is not None:
+                prologue()
+            fn()
+            if epilogue is not None:
+                epilogue()
+
+        # one call outside the capture first (one-time attribute set-up)
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            body()
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            body()
+        return g
 
     def out_f64(self) -> np.ndarray:
         return self.out.float().cpu().numpy().astype(np.float64)

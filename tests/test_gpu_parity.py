@@ -253,3 +253,30 @@ def test_zero_token_call_is_a_no_op():
     lib.reshape_and_cache(out[:, :2], out[:, :2], kc, kc,
                           torch.zeros(0, dtype=torch.int64, device=dev))
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_graph_replay_matches_direct_calls(d):
+    """A CUDA graph of the step (cache write + attention, the launches chained
+    as programmatic dependents) replays to the same bytes as direct calls, and
+    both match the oracle; so does a graph of the attention call alone."""
+    from paged_kv_cache_469_b200 import lib
+    from paged_kv_cache_469_b200.step import DeviceStep
+    step = random_step(71 + d, dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=d,
+                       num_seqs=8, max_ctx=900, max_q=300)
+    ds = DeviceStep(step)
+    ds.run()
+    torch.cuda.synchronize()
+    direct = _bits(ds.out).copy()
+    g_step = ds.capture("step")
+    g_attn = ds.capture("attention")
+    for g in (g_step, g_attn, g_step):
+        ds.out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert _bits(ds.out).tobytes() == direct.tobytes()
+    assert lib.workspace_status(ds.workspace) == 0
+    st = oracle_state(step)
+    assert _bits(ds.k_cache).tobytes() == st["k_cache"].tobytes()
+    assert_close(ds.out_f64(), oracle_outputs(step, st, num_threads=NTHREADS), "bf16",
+                 "graph replay")
