@@ -161,6 +161,35 @@ int pa_attention_varlen(void* out, const void* q, const void* k_cache, const voi
                         struct CUstream_st* stream);
 
 /*
+ * pa_attention_varlen_write_cache -- pa_reshape_and_cache of the step's new
+ * tokens followed by pa_attention_varlen, in one call.  (The pages describe
+ * the two operations one after the other; this call gives the same results.)
+ *
+ * Arguments: those of pa_attention_varlen, plus the new rows k_new, v_new
+ * ([num_tokens][num_kv_heads][head_dim], 16-byte aligned) and slot_mapping
+ * (int64 [num_tokens]) as pa_reshape_and_cache takes them; k_cache and
+ * v_cache are written.  Results: the cache bytes of pa_reshape_and_cache and
+ * the output of pa_attention_varlen on the updated cache.
+ *
+ * When every sequence of the step is decode-class (bf16), the decode kernel
+ * writes the rows itself: each CTA first stores the new tokens that fall in
+ * its own range of its sequence's keys, then reads them back through the
+ * block table.  One launch instead of two.  This requires the usual layout of
+ * a step: a token's slot is the slot of its own position in its own
+ * sequence's block table (block_tables[s][pos / 16] * 16 + pos % 16), and no
+ * other sequence of the step reads that slot.  Otherwise (prefill chunks, or
+ * fp32) the cache write runs as its own kernel first.
+ */
+int pa_attention_varlen_write_cache(
+    void* out, const void* q, const void* k_new, const void* v_new, void* k_cache,
+    void* v_cache, const int64_t* slot_mapping, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* seq_lens, const int32_t* query_start_loc,
+    int num_seqs, int num_tokens, int max_query_len, int max_seq_len, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+    void* workspace, size_t workspace_bytes, const int32_t* seq_lens_host,
+    const int32_t* query_start_loc_host, struct CUstream_st* stream);
+
+/*
  * pa_attention_varlen_static_scratch -- pa_attention_varlen for callers that
  * cannot allocate device memory.  (The pages describe no such call; it has no
  * counterpart in the method itself.)

@@ -111,7 +111,7 @@ struct DecodeSmem {
   static constexpr int kSlotBytes = 2 * kTileBytes;      // K tile + V tile
 };
 
-template <int D, bool kRows16, int kStages, int kWarps>
+template <int D, bool kRows16, int kStages, int kWarps, bool kWriteCache>
 __global__ void __launch_bounds__(kWarps * 32)
 decode_splitk_kernel(const AttnParams p) {
   constexpr int NJ = D / 32;  // 16-byte K chunks per key row a lane reads
@@ -151,10 +151,45 @@ decode_splitk_kernel(const AttnParams p) {
   if (part >= nparts || nparts > p.max_parts || L > p.max_seq_len ||
       (L + kBlockSize - 1) / kBlockSize > p.max_blocks_per_seq)
     return;
-  const int t_begin = part * P;
-  const int t_end = min(L, t_begin + P);
-  const int blk_begin = t_begin / kBlockSize;
-  const int blk_end = (t_end + kBlockSize - 1) / kBlockSize;
+  // nparts partitions of equal whole blocks (the last may be shorter; with
+  // partitions of at least 32 blocks none is empty for up to 32 partitions,
+  // and an empty one still reports (max -inf, sum 0) to the merge)
+  const int nblk_seq = (L + kBlockSize - 1) / kBlockSize;
+  const int pblk = (nblk_seq + nparts - 1) / nparts;
+  const int blk_begin = part * pblk;
+  const int blk_end = min(nblk_seq, blk_begin + pblk);
+
+  if constexpr (kWriteCache) {
+    // This step's new tokens of the sequence that fall in this partition's
+    // key range go into their cache slots first (as pa_reshape_and_cache
+    // would); only this CTA reads those keys of this kv-head, after the fence
+    // and the barrier below.
+    const int lo = max(L - ql, blk_begin * kBlockSize), hi = min(L, blk_end * kBlockSize);
+    if (hi > lo) {
+      constexpr int kVec = D * 2 / 16;  // 16-byte vectors per row
+      const int n = (hi - lo) * kVec;
+      const int64_t num_slots = (int64_t)p.num_blocks * kBlockSize;
+      const uint4* kn = (const uint4*)p.k_new;
+      const uint4* vn = (const uint4*)p.v_new;
+      uint4* kcw = (uint4*)const_cast<void*>(p.k_cache);
+      uint4* vcw = (uint4*)const_cast<void*>(p.v_cache);
+      for (int i = threadIdx.x; i < 2 * n; i += blockDim.x) {
+        const bool is_v = i >= n;
+        const int ii = is_v ? i - n : i;
+        const int j = ii / kVec, c = ii % kVec;
+        const int tok = q0 + (lo - (L - ql)) + j;
+        const int64_t slot = p.slot_mapping[tok];
+        if (slot < 0 || slot >= num_slots) continue;  // padding / out-of-pool slot
+        const int64_t dst =
+            ((slot / kBlockSize * p.num_kv_heads + kvh) * kBlockSize + slot % kBlockSize) * kVec + c;
+        const int64_t src = ((int64_t)tok * p.num_kv_heads + kvh) * kVec + c;
+        if (is_v) vcw[dst] = vn[src];
+        else kcw[dst] = kn[src];
+      }
+      __threadfence();
+    }
+    __syncthreads();
+  }
 
   // ---- this warp's block ids, one per lane (lane i <-> i-th block of the warp)
   const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks_per_seq;
@@ -452,10 +487,10 @@ decode_splitk_kernel(const AttnParams p) {
   if (threadIdx.x == 0) p.ws_counter[unit] = 0;  // ready for the next call
 }
 
-template <int D, bool kRows16, int kStages>
+template <int D, bool kRows16, int kStages, bool kWriteCache>
 cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
   constexpr int kWarps = kDecodeWarps;
-  auto kernel = decode_splitk_kernel<D, kRows16, kStages, kWarps>;
+  auto kernel = decode_splitk_kernel<D, kRows16, kStages, kWarps, kWriteCache>;
   const int ring = kWarps * kStages * DecodeSmem<D>::kSlotBytes;
   const int merge = kWarps * kDecodeRows * D * (int)sizeof(float);
   // the cross-partition merge: (max, sum) per partition and row, 1 / sum per row
@@ -466,7 +501,8 @@ cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
   cudaError_t e = raise_smem_limit(kernel, smem, smem_done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.max_parts, p.num_kv_heads, p.num_seqs);
+  const int parts = (p.max_seq_len + p.part_tokens - 1) / p.part_tokens;  // <= p.max_parts
+  cfg.gridDim = dim3(parts > 0 ? parts : 1, p.num_kv_heads, p.num_seqs);
   cfg.blockDim = dim3(kWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -478,7 +514,37 @@ cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
+template <int D, bool kRows16, int kStages>
+int wave_ctas_one() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  constexpr int kWarps = kDecodeWarps;
+  const int ring = kWarps * kStages * DecodeSmem<D>::kSlotBytes;
+  const int merge = kWarps * kDecodeRows * D * (int)sizeof(float);
+  int per_sm = 0, sms = 0;
+  auto kernel = decode_splitk_kernel<D, kRows16, kStages, kWarps, false>;
+  static std::atomic<int> smem_done[64];
+  raise_smem_limit(kernel, ring > merge ? ring : merge, smem_done);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kWarps * 32,
+                                                    ring > merge ? ring : merge) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 2 * 148;
+  n = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 148);
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 }  // namespace
+
+int decode_wave_ctas(int head_dim, int rows) {
+  constexpr int s64 = PA_DECODE_STAGES_D64, s128 = PA_DECODE_STAGES_D128;
+  if (head_dim == 64)
+    return rows > 8 ? wave_ctas_one<64, true, s64>() : wave_ctas_one<64, false, s64>();
+  return rows > 8 ? wave_ctas_one<128, true, s128>() : wave_ctas_one<128, false, s128>();
+}
 
 cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
                                  cudaStream_t stream) {
@@ -487,10 +553,17 @@ cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_quer
   const bool rows16 = max_rows > 8;
   cudaError_t e;
   constexpr int s64 = PA_DECODE_STAGES_D64, s128 = PA_DECODE_STAGES_D128;
+  const bool wc = p.slot_mapping != nullptr;
   if (head_dim == 64)
-    e = rows16 ? launch_one<64, true, s64>(p, stream) : launch_one<64, false, s64>(p, stream);
+    e = rows16 ? (wc ? launch_one<64, true, s64, true>(p, stream)
+                     : launch_one<64, true, s64, false>(p, stream))
+               : (wc ? launch_one<64, false, s64, true>(p, stream)
+                     : launch_one<64, false, s64, false>(p, stream));
   else
-    e = rows16 ? launch_one<128, true, s128>(p, stream) : launch_one<128, false, s128>(p, stream);
+    e = rows16 ? (wc ? launch_one<128, true, s128, true>(p, stream)
+                     : launch_one<128, true, s128, false>(p, stream))
+               : (wc ? launch_one<128, false, s128, true>(p, stream)
+                     : launch_one<128, false, s128, false>(p, stream));
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

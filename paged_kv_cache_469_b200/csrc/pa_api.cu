@@ -9,32 +9,42 @@ namespace pa {
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Keys per split-K partition: the largest power of two in [PA_PART_MIN,
-// PA_PART_MAX] that still gives the GPU about PA_TARGET_CTAS CTAs when the
-// sequences average half of max_seq_len.  Hardware CTA scheduling then spreads
-// the partitions over the SMs as they free up.
+// Split-K partitions.  The workspace is laid out for partitions as short as
+// part_tokens_floor(max_seq_len) keys: a power of two in [PA_PART_MIN,
+// PA_PART_MAX], at least a quarter of max_seq_len, so that a sequence never
+// needs more than four partitions unless it is longer than 4 * PA_PART_MAX.
+// Each call then picks its own partition length, no shorter than that floor
+// and no longer than PA_PART_MAX: about the step's total keys divided by the
+// number of decode CTAs the GPU holds at once (one full wave; the hardware
+// hands later partitions to SMs as they free up), so that a small step still
+// keeps every SM streaming and no partition is much longer than the rest.
 #ifndef PA_PART_MIN
-#define PA_PART_MIN 1024
+#define PA_PART_MIN 512
 #endif
 #ifndef PA_PART_MAX
 #define PA_PART_MAX 2048
 #endif
-#ifndef PA_TARGET_CTAS
-#define PA_TARGET_CTAS (8 * 148)
-#endif
-static int choose_part_tokens(int num_seqs, int num_kv_heads, int max_seq_len) {
-  const long units = (long)num_seqs * num_kv_heads;
-  int part = PA_PART_MAX;
-  while (part > PA_PART_MIN &&
-         units * (((long)max_seq_len / 2 + part - 1) / part) < (long)PA_TARGET_CTAS)
-    part /= 2;
+static int part_tokens_floor(int max_seq_len) {
+  int part = PA_PART_MIN;
+  while (part < PA_PART_MAX && (long)part * 4 < (long)max_seq_len) part *= 2;
   return part;
+}
+#ifndef PA_DECODE_WAVES
+#define PA_DECODE_WAVES 0.5
+#endif
+static int part_tokens_for_step(long total_unit_keys, int wave_ctas, int floor_tokens) {
+  const long ctas = (long)(PA_DECODE_WAVES * (wave_ctas > 0 ? wave_ctas : 1)) + 1;
+  long part = (total_unit_keys + ctas - 1) / ctas;
+  part = (part + kBlockSize - 1) / kBlockSize * kBlockSize;
+  if (part < floor_tokens) part = floor_tokens;
+  if (part > PA_PART_MAX) part = PA_PART_MAX;
+  return (int)part;
 }
 
 WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_seq_len) {
   WorkspaceLayout w{};
-  w.part_tokens = choose_part_tokens(num_seqs, num_kv_heads, max_seq_len);
+  w.part_tokens = part_tokens_floor(max_seq_len);
   w.max_parts = max(1, (max_seq_len + w.part_tokens - 1) / w.part_tokens);
   // prefill items: at most ceil(q_len / 128) <= ceil(max_seq_len / 128) per sequence and q-head
   const long items = (long)num_seqs * ((max_seq_len + kPrefillQTile - 1) / kPrefillQTile) *
@@ -113,16 +123,25 @@ extern "C" int pa_workspace_init(void* workspace, size_t workspace_bytes,
              : PA_ERR_CUDA;
 }
 
-extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache,
-                                   const void* v_cache, const int32_t* block_tables,
-                                   int max_blocks_per_seq, const int32_t* seq_lens,
-                                   const int32_t* query_start_loc, int num_seqs, int num_tokens,
-                                   int max_query_len, int max_seq_len, int num_q_heads,
-                                   int num_kv_heads, int head_dim, int block_size,
-                                   int num_blocks, float scale, pa_dtype dtype, void* workspace,
-                                   size_t workspace_bytes, const int32_t* seq_lens_host,
-                                   const int32_t* query_start_loc_host,
-                                   struct CUstream_st* stream) {
+namespace {
+
+// The new tokens' K/V rows a call writes into the cache before it reads it
+// (pa_attention_varlen_write_cache); all null for pa_attention_varlen.
+struct CacheWrite {
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  const int64_t* slot_mapping = nullptr;
+};
+
+int attention_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+                   const int32_t* query_start_loc, int num_seqs, int num_tokens,
+                   int max_query_len, int max_seq_len, int num_q_heads, int num_kv_heads,
+                   int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+                   void* workspace, size_t workspace_bytes, const int32_t* seq_lens_host,
+                   const int32_t* query_start_loc_host, struct CUstream_st* stream,
+                   const CacheWrite& cw) {
+  const bool write_cache = cw.slot_mapping != nullptr;
   // ---- scalar checks
   if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || max_seq_len < 0 ||
       num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks < 0 || max_blocks_per_seq < 0)
@@ -140,15 +159,19 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
     return PA_ERR_INVALID;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
+  if (write_cache && (!cw.k_new || !cw.v_new || !aligned16(cw.k_new) || !aligned16(cw.v_new)))
+    return PA_ERR_INVALID;
 
   // ---- optional host copies: check the step and see which kernels it needs
   bool any_decode = true, any_prefill = true;
   int prefill_items = -1;  // unknown without the host copies
+  long decode_keys = -1;   // sum of the decode-class sequences' lengths, when known
   if (seq_lens_host && query_start_loc_host) {
     if (query_start_loc_host[0] != 0 || query_start_loc_host[num_seqs] != num_tokens)
       return PA_ERR_INVALID;
     any_decode = any_prefill = false;
     prefill_items = 0;
+    decode_keys = 0;
     for (int s = 0; s < num_seqs; ++s) {
       const int ql = query_start_loc_host[s + 1] - query_start_loc_host[s];
       const int L = seq_lens_host[s];
@@ -156,6 +179,7 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
       if (ql == 0) continue;
       if (ql * group <= kDecodeRows) {
         any_decode = true;
+        decode_keys += L;
       } else {
         any_prefill = true;
         prefill_items += (ql + kPrefillQTile - 1) / kPrefillQTile * num_q_heads;
@@ -178,8 +202,13 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
   p.query_start_loc = query_start_loc;
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.max_seq_len = max_seq_len;
-  p.part_tokens = w.part_tokens;
-  p.max_parts = w.max_parts;
+  p.max_parts = w.max_parts;  // the workspace's partitions per (sequence, kv-head)
+  {
+    const long keys = decode_keys >= 0 ? decode_keys : (long)num_seqs * (max_seq_len / 2 + 1);
+    const int rows = min(max_query_len * group, kDecodeRows);
+    p.part_tokens = part_tokens_for_step(keys * num_kv_heads,
+                                         decode_wave_ctas(head_dim, rows), w.part_tokens);
+  }
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;
   p.num_q_heads = num_q_heads;
@@ -189,13 +218,29 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = (cudaStream_t)stream;
+  const int elem_bytes = dtype == PA_DTYPE_F32 ? 4 : 2;
+  // The decode kernel writes a sequence's new rows itself (each CTA those
+  // that fall in its own key range, before it reads them back) when every
+  // sequence of the step is decode-class; otherwise the cache write runs as
+  // its own kernel first, since a prefill chunk's tiles need all of its rows.
+  const bool fused_write = write_cache && dtype == PA_DTYPE_BF16 && !any_prefill;
+  // every argument check comes before the first launch
+  if (dtype != PA_DTYPE_F32 &&
+      (!workspace || workspace_bytes < w.total || !aligned16(workspace)))
+    return PA_ERR_INVALID;
+  if (write_cache && !fused_write) {
+    cudaError_t e = launch_reshape_and_cache(cw.k_new, cw.v_new, const_cast<void*>(k_cache),
+                                             const_cast<void*>(v_cache), cw.slot_mapping,
+                                             num_tokens, num_kv_heads, head_dim, num_blocks,
+                                             elem_bytes, st);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+  }
 
   if (dtype == PA_DTYPE_F32) {
     cudaError_t e = launch_attention_simple(p, head_dim, false, 0, st);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
 
-  if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return PA_ERR_INVALID;
   char* ws = (char*)workspace;
   p.ws_status = (int*)(ws + w.status_off);
   p.ws_counter = (int*)(ws + w.counter_off);
@@ -203,6 +248,11 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
   p.ws_ml = (float*)(ws + w.ml_off);
   p.ws_items = (int4*)(ws + w.items_off);
   p.max_items = w.max_items;
+  if (fused_write) {
+    p.k_new = cw.k_new;
+    p.v_new = cw.v_new;
+    p.slot_mapping = cw.slot_mapping;
+  }
   if (any_decode) {
     cudaError_t e = launch_decode_splitk(p, head_dim, max_query_len, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;
@@ -212,4 +262,43 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   int max_blocks_per_seq, const int32_t* seq_lens,
+                                   const int32_t* query_start_loc, int num_seqs, int num_tokens,
+                                   int max_query_len, int max_seq_len, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int num_blocks, float scale, pa_dtype dtype, void* workspace,
+                                   size_t workspace_bytes, const int32_t* seq_lens_host,
+                                   const int32_t* query_start_loc_host,
+                                   struct CUstream_st* stream) {
+  return attention_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                        query_start_loc, num_seqs, num_tokens, max_query_len, max_seq_len,
+                        num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
+                        workspace, workspace_bytes, seq_lens_host, query_start_loc_host, stream,
+                        CacheWrite{});
+}
+
+extern "C" int pa_attention_varlen_write_cache(
+    void* out, const void* q, const void* k_new, const void* v_new, void* k_cache,
+    void* v_cache, const int64_t* slot_mapping, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* seq_lens, const int32_t* query_start_loc,
+    int num_seqs, int num_tokens, int max_query_len, int max_seq_len, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+    void* workspace, size_t workspace_bytes, const int32_t* seq_lens_host,
+    const int32_t* query_start_loc_host, struct CUstream_st* stream) {
+  if (!slot_mapping && num_tokens > 0) return PA_ERR_INVALID;
+  CacheWrite cw;
+  cw.k_new = k_new;
+  cw.v_new = v_new;
+  cw.slot_mapping = slot_mapping;
+  return attention_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                        query_start_loc, num_seqs, num_tokens, max_query_len, max_seq_len,
+                        num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
+                        workspace, workspace_bytes, seq_lens_host, query_start_loc_host, stream,
+                        slot_mapping ? cw : CacheWrite{});
 }

@@ -61,7 +61,14 @@ struct AttnParams {
   float scale;       // softmax scale (natural-log base)
   float scale_log2;  // scale * log2(e), for exp2-based softmax
   // split-K decode
-  int part_tokens;   // keys per partition (multiple of 16)
+  // decode-class steps of pa_attention_varlen_write_cache: the new tokens' K/V
+  // rows [num_tokens][Hkv][D] and their slots, written by the decode kernel
+  // (null otherwise)
+  const void* k_new;
+  const void* v_new;
+  const int64_t* slot_mapping;
+  int part_tokens;   // keys per partition at most (multiple of 16); a sequence is cut
+                     // into ceil(L / part_tokens) partitions of equal whole blocks
   int max_parts;     // partitions the workspace holds per (sequence, kv-head)
   float* ws_o;       // [num_seqs*Hkv][max_parts][16][D] unnormalised partial outputs
   float* ws_ml;      // [num_seqs*Hkv][max_parts][16][2] running max (log2 units), sum
@@ -97,6 +104,9 @@ cudaError_t launch_attention_simple(const AttnParams& p, int head_dim, bool is_b
                                     int min_rows_per_kv_head, cudaStream_t stream);
 
 // Split-K decode kernel (bf16): sequences with q_len * group <= 16.
+// Decode CTAs the GPU holds at once for this head_dim and query-row count
+// (SMs x resident CTAs per SM); looked up once per device and shape.
+int decode_wave_ctas(int head_dim, int rows);
 cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
                                  cudaStream_t stream);
 

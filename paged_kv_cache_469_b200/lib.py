@@ -21,7 +21,7 @@ PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
 # every symbol include/pa.h declares
 EXPORTS = ("pa_status_string", "pa_reshape_and_cache", "pa_attention_workspace_size",
            "pa_workspace_init", "pa_workspace_status", "pa_attention_varlen",
-           "pa_attention_varlen_static_scratch")
+           "pa_attention_varlen_write_cache", "pa_attention_varlen_static_scratch")
 
 _lib = None
 
@@ -56,6 +56,10 @@ def library() -> ctypes.CDLL:
         lib.pa_attention_varlen.argtypes = [c_p, c_p, c_p, c_p, c_p, c_int, c_p, c_p, c_int,
                                             c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                             c_int, c_f, c_int, c_p, c_sz, c_p, c_p, c_p]
+        lib.pa_attention_varlen_write_cache.restype = c_int
+        lib.pa_attention_varlen_write_cache.argtypes = [
+            c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_int, c_p, c_p, c_int, c_int, c_int, c_int,
+            c_int, c_int, c_int, c_int, c_int, c_f, c_int, c_p, c_sz, c_p, c_p, c_p]
         _lib = lib
     return _lib
 
@@ -157,4 +161,38 @@ def attention_varlen(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     del sl_keep, qs_keep
     if rc != PA_OK:
         raise PAError(rc, "pa_attention_varlen")
+    return out
+
+
+def attention_varlen_write_cache(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor,
+                                 v_new: torch.Tensor, k_cache: torch.Tensor,
+                                 v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                                 block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                 query_start_loc: torch.Tensor, *, max_query_len: int,
+                                 max_seq_len: int, scale: float, workspace: torch.Tensor | None,
+                                 seq_lens_host=None, query_start_loc_host=None,
+                                 stream=None) -> torch.Tensor:
+    """The step's cache write and attention in one call (see
+    pa_attention_varlen_write_cache in pa.h)."""
+    num_blocks, hkv, bs, d = k_cache.shape
+    t, hq, _ = q.shape
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32 or \
+            query_start_loc.dtype != torch.int32:
+        raise TypeError("block_tables, seq_lens and query_start_loc must be int32")
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    sl_ptr, sl_keep = _host_i32(seq_lens_host)
+    qs_ptr, qs_keep = _host_i32(query_start_loc_host)
+    ws_ptr, ws_n = (0, 0) if workspace is None else (_dev(workspace, "workspace"),
+                                                     workspace.numel() * workspace.element_size())
+    rc = library().pa_attention_varlen_write_cache(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_new, "k_new"), _dev(v_new, "v_new"),
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(slot_mapping, "slot_mapping"),
+        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(seq_lens, "seq_lens"),
+        _dev(query_start_loc, "query_start_loc"), seq_lens.shape[0], t, max_query_len,
+        max_seq_len, hq, hkv, d, bs, num_blocks, float(scale), _dtype_code(q), ws_ptr, ws_n,
+        sl_ptr, qs_ptr, _stream(stream))
+    del sl_keep, qs_keep
+    if rc != PA_OK:
+        raise PAError(rc, "pa_attention_varlen_write_cache")
     return out

@@ -77,17 +77,29 @@ class DeviceStep:
             query_start_loc_host=p.query_start_loc if host_hints else None, stream=stream)
 
     def run(self, stream=None, host_hints: bool = True) -> torch.Tensor:
-        """One step: cache write of the new tokens, then attention."""
+        """One step: cache write of the new tokens, then attention (two calls)."""
         self.write_new_tokens(stream)
         return self.attention(stream, host_hints)
 
+    def run_fused(self, stream=None, host_hints: bool = True) -> torch.Tensor:
+        """One step as a single pa_attention_varlen_write_cache call."""
+        p = self.plan
+        return lib.attention_varlen_write_cache(
+            self.out, self.q, self.k_new, self.v_new, self.k_cache, self.v_cache,
+            self.slot_mapping, self.block_tables, self.seq_lens, self.query_start_loc,
+            max_query_len=p.max_query_len, max_seq_len=p.max_seq_len, scale=self.step.scale,
+            workspace=self.workspace, seq_lens_host=p.seq_lens if host_hints else None,
+            query_start_loc_host=p.query_start_loc if host_hints else None, stream=stream)
+
     def capture(self, what: str = "step", prologue=None, epilogue=None) -> torch.cuda.CUDAGraph:
         """A CUDA graph of this step's launches: "step" (cache write of the new
-        tokens, then attention) or "attention" (the attention call alone).
+        tokens, then attention), "fused" (the same as one
+        pa_attention_varlen_write_cache call) or "attention" (the attention
+        call alone).
         ``prologue`` / ``epilogue`` are captured before / after them (for
         example host-device copies).  Replaying the graph repeats the step on
         whatever the step's device tensors hold at that time."""
-        fn = self.run if what == "step" else self.attention
+        fn = {"step": self.run, "fused": self.run_fused, "attention": self.attention}[what]
 
         def body():
             if prologue is not None:

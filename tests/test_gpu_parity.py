@@ -280,3 +280,71 @@ def test_graph_replay_matches_direct_calls(d):
     assert _bits(ds.k_cache).tobytes() == st["k_cache"].tobytes()
     assert_close(ds.out_f64(), oracle_outputs(step, st, num_threads=NTHREADS), "bf16",
                  "graph replay")
+
+
+def _fused_check(step, host_hints=True, d_dtype="bf16"):
+    from paged_kv_cache_469_b200 import lib
+    from paged_kv_cache_469_b200.step import DeviceStep
+    ds = DeviceStep(step)
+    ds.run_fused(host_hints=host_hints)
+    torch.cuda.synchronize()
+    if step.dtype == "bf16":
+        assert lib.workspace_status(ds.workspace) == 0
+    st = oracle_state(step)
+    assert _bits(ds.k_cache).tobytes() == st["k_cache"].tobytes(), "k_cache differs"
+    assert _bits(ds.v_cache).tobytes() == st["v_cache"].tobytes(), "v_cache differs"
+    assert_close(ds.out_f64(), oracle_outputs(step, st, num_threads=NTHREADS), step.dtype,
+                 step.name + " (one call)")
+    n = step.num_seqs * step.num_kv_heads * 4
+    assert int(ds.workspace[256:256 + n].count_nonzero()) == 0
+    return ds
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv,ql", [(32, 4, 1), (32, 8, 2), (8, 8, 16), (16, 1, 1)])
+@pytest.mark.parametrize("hints", [True, False])
+def test_write_cache_call_decode_steps(d, hq, hkv, ql, hints):
+    """Decode-class steps: the decode kernel writes the new rows itself (new
+    tokens crossing block and partition boundaries included); cache bytes and
+    outputs equal the two-call path's and the oracle's."""
+    rng = np.random.default_rng(1000 + d + hq + ql)
+    lens = rng.integers(ql, 3000, size=12)
+    lens[0], lens[1] = 17, ql  # a token at a block's start; a sequence of only new tokens
+    step = make_step(name="fused_decode", dtype="bf16", num_q_heads=hq, num_kv_heads=hkv,
+                     head_dim=d, num_blocks=int(np.sum((lens + 15) // 16)) + 40,
+                     seq_lens=lens, query_lens=np.full(12, ql), seed=77)
+    ds = _fused_check(step, host_hints=hints)
+    if hints:  # the same partitioning as the two-call path: the same bytes
+        two = DeviceStepTwoCall(step)
+        assert _bits(two.out).tobytes() == _bits(ds.out).tobytes()
+
+
+def DeviceStepTwoCall(step):
+    from paged_kv_cache_469_b200.step import DeviceStep
+    ds = DeviceStep(step)
+    ds.run()
+    torch.cuda.synchronize()
+    return ds
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_write_cache_call_mixed_and_fp32_steps(d):
+    """Steps with prefill chunks (and fp32 steps) take the write-then-attend
+    order inside the one call."""
+    _fused_check(random_step(91 + d, dtype="bf16", num_q_heads=8, num_kv_heads=2, head_dim=d,
+                             num_seqs=5, max_ctx=400, max_q=200))
+    _fused_check(random_step(93 + d, dtype="f32", num_q_heads=4, num_kv_heads=4, head_dim=d,
+                             num_seqs=3, max_ctx=60, max_q=20))
+
+
+def test_write_cache_call_graph_replay():
+    from paged_kv_cache_469_b200.step import DeviceStep
+    step = workload("decode_tinyllama")
+    ds = DeviceStep(step)
+    g = ds.capture("fused")
+    ds.out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    got = _bits(ds.out).copy()
+    ref = DeviceStepTwoCall(step)
+    assert got.tobytes() == _bits(ref.out).tobytes()
