@@ -348,3 +348,28 @@ def test_write_cache_call_graph_replay():
     got = _bits(ds.out).copy()
     ref = DeviceStepTwoCall(step)
     assert got.tobytes() == _bits(ref.out).tobytes()
+
+
+@pytest.mark.parametrize("case", ["one_long_unit", "many_tiny_units", "mixed_with_prefill"])
+@pytest.mark.parametrize("hints", [True, False])
+def test_decode_partition_edge_steps(case, hints):
+    """Split-K decode on edge-shaped steps, with the partition length taken
+    from the host copies or estimated without them: one long unit split into
+    several partitions, hundreds of one- and two-block units, and decode units
+    mixed with a prefill chunk."""
+    if case == "one_long_unit":
+        step = make_step(name=case, dtype="bf16", num_q_heads=8, num_kv_heads=1, head_dim=128,
+                         num_blocks=260, seq_lens=[3000], query_lens=[1], seed=5)
+    elif case == "many_tiny_units":
+        lens = np.random.default_rng(3).integers(1, 40, size=300)
+        step = make_step(name=case, dtype="bf16", num_q_heads=32, num_kv_heads=4, head_dim=64,
+                         num_blocks=int(np.sum((lens + 15) // 16)) + 10, seq_lens=lens,
+                         query_lens=np.ones(300, np.int32), seed=6)
+    else:
+        step = random_step(97, dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                           num_seqs=10, max_ctx=1500, max_q=3)
+        step = make_step(name=case, dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
+                         num_blocks=step.num_blocks + 64,
+                         seq_lens=np.concatenate([step.seq_lens, [700]]),
+                         query_lens=np.concatenate([step.query_lens, [300]]), seed=7)
+    run_and_check(step, host_hints=hints)
