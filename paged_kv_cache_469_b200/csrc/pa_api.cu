@@ -258,7 +258,8 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
   if (any_prefill) {
-    cudaError_t e = launch_prefill_tcgen05(p, head_dim, max_query_len, prefill_items, st);
+    cudaError_t e = launch_prefill_tcgen05(p, head_dim, max_query_len, prefill_items,
+                                           seq_lens_host, query_start_loc_host, st);
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;

@@ -116,6 +116,7 @@ cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_quer
 constexpr int kPrefillQTile = 128;  // query rows per Q tile (MMA M); a work item holds two
 constexpr int kPrefillKvTile = 128;  // keys per pipeline step
 cudaError_t launch_prefill_tcgen05(const AttnParams& p, int head_dim, int max_query_len,
-                                   int num_items, cudaStream_t stream);
+                                   int num_items, const int32_t* seq_lens_host,
+                                   const int32_t* query_start_loc_host, cudaStream_t stream);
 
 }  // namespace pa

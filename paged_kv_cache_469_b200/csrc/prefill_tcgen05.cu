@@ -309,8 +309,19 @@ struct ItemInfo {
   int q0, ql, L;
 };
 
-__device__ __forceinline__ ItemInfo load_item(const AttnParams& p, int w) {
-  const int4 it = p.ws_items[1 + w];
+// A work list the host built from its copies of the step's lengths, passed as
+// a kernel parameter (count 0: the list is in the workspace, built by
+// prefill_plan_kernel).
+constexpr int kParamItems = 1024;
+struct PrefillWork {
+  int count;
+  int pad[3];
+  int4 items[kParamItems];
+};
+
+__device__ __forceinline__ ItemInfo load_item(const AttnParams& p, const PrefillWork& work,
+                                              int w) {
+  const int4 it = work.count > 0 ? work.items[w] : p.ws_items[1 + w];
   ItemInfo r;
   r.seq = it.x; r.qt0 = it.y; r.head0 = it.z; r.ntiles = it.w;
   r.q0 = p.query_start_loc[r.seq];
@@ -329,7 +340,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, int pair_heads) {
+                       const __grid_constant__ CUtensorMap tm_v, int pair_heads,
+                       const __grid_constant__ PrefillWork work) {
   using LY = PrefillLayout<D>;
   constexpr int kPanels = LY::kPanels;
   extern __shared__ unsigned char smem_raw[];
@@ -379,7 +391,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
   // this grid before it reads anything)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int num_items = p.ws_items[0].x;
+  const int num_items = work.count > 0 ? work.count : p.ws_items[0].x;
   int* status = p.ws_status;
 
   if (warp >= 8) {
@@ -395,7 +407,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       for (int k = 0; ok; ++k) {
         const int w = item_index(k);
         if (w >= num_items) break;
-        const ItemInfo it = load_item(p, w);
+        const ItemInfo it = load_item(p, work, w);
         const int kvh = it.head0 / p.group;
         const int nblk = (it.L + kBlockSize - 1) / kBlockSize;
         const int shift = nblk * kBlockSize - it.L;  // unwritten slots of the last block
@@ -497,7 +509,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
       for (int k = 0; ok; ++k) {
         const int w = item_index(k);
         if (w >= num_items) break;
-        const ItemInfo it = load_item(p, w);
+        const ItemInfo it = load_item(p, work, w);
         ok = wait_bar(bar(kBarQFull), k & 1, abort_flag, status);
         const uint32_t g_first = g;
         for (int t = 0; t < it.ntiles && ok; ++t, ++g) {
@@ -543,7 +555,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
     for (int k = 0; ok; ++k) {
       const int w = item_index(k);
       if (w >= num_items) break;
-      const ItemInfo it = load_item(p, w);
+      const ItemInfo it = load_item(p, work, w);
       const int head = pair_heads ? it.head0 + h : it.head0;
       const int qt = pair_heads ? it.qt0 : it.qt0 + h;
       const int jq = qt * QT + row;
@@ -712,8 +724,8 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
 // store the count in ws_items[0].x.  An item pairs two q-heads of one kv-head
 // (pair_heads: the group is even) or two consecutive query tiles of one
 // q-head; its tile count covers the later of its two query tiles.
-__device__ __forceinline__ void prefill_item_range(int L, int ql, int pair_heads, int i,
-                                                   int* last_row_pos) {
+__host__ __device__ __forceinline__ void prefill_item_range(int L, int ql, int pair_heads,
+                                                            int i, int* last_row_pos) {
   const int hi_tile = pair_heads ? i : 2 * i + 1;
   const int last_row = min((hi_tile + 1) * QT, ql) - 1;
   *last_row_pos = L - ql + last_row;
@@ -811,8 +823,52 @@ int sm_count() {
   return n[dev] > 0 ? n[dev] : 148;
 }
 
+// The work list of prefill_plan_kernel, built on the host from its copies of
+// the step's lengths: the same items, heaviest first.  False when there are
+// more items than a kernel parameter holds.
+bool host_work_list(PrefillWork* work, const AttnParams& p, const int32_t* seq_lens_host,
+                    const int32_t* query_start_loc_host, int max_tiles, int pair_heads) {
+  const int per_tile = pair_heads ? p.num_q_heads / 2 : p.num_q_heads;
+  static thread_local int hist[1 << 16];
+  if (max_tiles + 1 > (1 << 16)) return false;
+  for (int i = 0; i <= max_tiles; ++i) hist[i] = 0;
+  long total = 0;
+  auto for_each_item = [&](auto fn) {
+    for (int s = 0; s < p.num_seqs; ++s) {
+      const int ql = query_start_loc_host[s + 1] - query_start_loc_host[s];
+      const int L = seq_lens_host[s];
+      if (ql * p.group <= kDecodeRows || ql > L) continue;
+      const int nq = (ql + QT - 1) / QT;
+      const int ni = pair_heads ? nq : (nq + 1) / 2;
+      for (int i = 0; i < ni; ++i) {
+        int last;
+        prefill_item_range(L, ql, pair_heads, i, &last);
+        fn(s, i, min(last / KT + 1, max_tiles));
+      }
+    }
+  };
+  for_each_item([&](int, int, int nt) { hist[nt] += per_tile; total += per_tile; });
+  if (total > kParamItems || total > p.max_items) return false;
+  int run = 0;
+  for (int nt = max_tiles; nt >= 0; --nt) {
+    const int c = hist[nt];
+    hist[nt] = run;
+    run += c;
+  }
+  for_each_item([&](int s, int i, int nt) {
+    int at = hist[nt];
+    hist[nt] += per_tile;
+    for (int h = 0; h < per_tile; ++h, ++at)
+      work->items[at] = pair_heads ? make_int4(s, i, 2 * h, nt) : make_int4(s, 2 * i, h, nt);
+  });
+  work->count = (int)total;
+  return total > 0;
+}
+
 template <int D>
-cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cudaStream_t stream) {
+cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items,
+                     const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
+                     cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, p.q, D, p.num_q_heads, p.num_tokens, (uint64_t)D * 2,
                 (uint64_t)p.num_q_heads * D * 2, 1, QT) ||
@@ -828,9 +884,14 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
 
-  // work list on the device
-  {
-    const int tiles = (p.max_blocks_per_seq * kBlockSize + KT - 1) / KT;
+  // the work list: from the host copies when given and small enough, else
+  // built on the device
+  static thread_local PrefillWork work;  // 16 KB: kept off the stack
+  const int tiles = (p.max_blocks_per_seq * kBlockSize + KT - 1) / KT;
+  work.count = 0;
+  if (!(seq_lens_host && query_start_loc_host &&
+        host_work_list(&work, p, seq_lens_host, query_start_loc_host, tiles, pair_heads))) {
+    work.count = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(1024);
@@ -847,7 +908,8 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
     cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_plan_kernel, p, tiles, pair_heads);
     if (e != cudaSuccess) return e;
   }
-  const int upper = num_items >= 0 ? num_items
+  const int upper = work.count > 0 ? work.count
+                  : num_items >= 0 ? num_items
                                    : (int)min((long)p.max_items,
                                               (long)p.num_seqs * ((max_query_len + QT - 1) / QT) *
                                                   p.num_q_heads);
@@ -864,15 +926,19 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items, cuda
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, pair_heads);
+  return cudaLaunchKernelEx(&cfg, kernel, p, tq, tk, tv, pair_heads, work);
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_tcgen05(const AttnParams& p, int head_dim, int max_query_len,
-                                   int num_items, cudaStream_t stream) {
-  cudaError_t e = head_dim == 64 ? launch_d<64>(p, max_query_len, num_items, stream)
-                                 : launch_d<128>(p, max_query_len, num_items, stream);
+                                   int num_items, const int32_t* seq_lens_host,
+                                   const int32_t* query_start_loc_host, cudaStream_t stream) {
+  cudaError_t e =
+      head_dim == 64
+          ? launch_d<64>(p, max_query_len, num_items, seq_lens_host, query_start_loc_host, stream)
+          : launch_d<128>(p, max_query_len, num_items, seq_lens_host, query_start_loc_host,
+                          stream);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
