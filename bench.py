@@ -38,10 +38,10 @@ WORKLOAD = "decode_tinyllama"
 MIXED_WORKLOAD = "mixed_llama3_8b"
 L2_BYTES = 126 * 1000 * 1000  # B200 L2, for sizing the rotation of workload copies
 MAX_COPIES = 8
-# dram__bytes_read.sum + dram__bytes_write.sum of one decode_splitk_kernel<64,0,4,4>
+# dram__bytes_read.sum + dram__bytes_write.sum of one decode_splitk_kernel<64,false,4,4,false>
 # launch on this workload, from an ncu --set full capture of that launch; set
 # to None whenever that kernel changes, until it is captured again
-DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_BYTES = 68_941_312 + 962_816
 
 
 def kv_bytes(step, seqs=None) -> int:
@@ -340,7 +340,8 @@ def bench_mixed(args, dev, stream, world, clocks):
                              "frac_of_bf16_sustained": round(
                                  tflops / peaks["bf16_tflops_sustained"], 4),
                              "peak_source": peaks["source"], "copies_rotated": pre_copies,
-                             "kernels": "prefill_plan_kernel + prefill_tcgen05_kernel<128>"}}
+                             "kernels": ("prefill_tcgen05_kernel<128> (work list from the "
+                                         "host copies of the step's lengths)")}}
 
 
 def bench_ours(args) -> None:
@@ -469,7 +470,7 @@ def bench_ours(args) -> None:
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": DECODE_TRAFFIC_BYTES, "traffic_unit": "bytes per launch (ncu)",
-                "kernel": "decode_splitk_kernel<64,0,4,4>",
+                "kernel": "decode_splitk_kernel<64,false,4,4,false> (attention call without the fused cache write)",
                 "peak_source": f"{peaks['source']} HBM copy bandwidth (burst)",
                 "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)}
     cpu = None

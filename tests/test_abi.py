@@ -88,6 +88,33 @@ def test_attention_argument_checks(L):
         palib.PA_ERR_INVALID
 
 
+def _varlen_wc(L, **kw):
+    args = dict(out=16, q=16, kn=16, vn=16, kc=16, vc=16, slots=16, bt=16, mb=8, sl=16, qsl=16,
+                S=1, T=1, mq=1, ms=16, hq=8, hkv=2, d=64, bs=16, nb=4, scale=0.125, dt=1, ws=0,
+                wsb=0, slh=None, qslh=None, stream=None)
+    args.update(kw)
+    return L.pa_attention_varlen_write_cache(*args.values())
+
+
+def test_write_cache_call_argument_checks(L):
+    """pa_attention_varlen_write_cache checks what pa_attention_varlen checks,
+    plus its new-row arguments, on the host, before any launch (and so before
+    any cache write)."""
+    assert _varlen_wc(L, d=96) == palib.PA_ERR_UNSUPPORTED
+    assert _varlen_wc(L, hkv=3) == palib.PA_ERR_INVALID
+    assert _varlen_wc(L, slots=0) == palib.PA_ERR_INVALID   # no slot mapping
+    assert _varlen_wc(L, kn=0) == palib.PA_ERR_INVALID      # no new K rows
+    assert _varlen_wc(L, vn=8) == palib.PA_ERR_INVALID      # misaligned new V rows
+    assert _varlen_wc(L, q=8) == palib.PA_ERR_INVALID
+    assert _varlen_wc(L, T=0) == palib.PA_OK                # nothing to do
+    import numpy as np
+    sl = np.array([4], np.int32)
+    ok_qsl = np.array([0, 1], np.int32)
+    # a decode step without a big enough workspace fails before the cache write
+    assert _varlen_wc(L, slh=sl.ctypes.data, qslh=ok_qsl.ctypes.data, ws=0, wsb=0) == \
+        palib.PA_ERR_INVALID
+
+
 def test_reshape_argument_checks(L):
     f = L.pa_reshape_and_cache
     assert f(16, 16, 16, 16, 16, 4, 2, 96, 16, 8, 1, None) == palib.PA_ERR_UNSUPPORTED
