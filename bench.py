@@ -410,34 +410,19 @@ def bench_ours(args) -> None:
     value = bytes_all / (step_ms_max / 1e3) / 1e9
 
     # ---- end to end through the public API from pinned host buffers: every step
-    # copies its inputs in, runs, and copies its output back
+    # copies its inputs in (one copy: the step's inputs are packed into one
+    # buffer on both sides), runs, and copies its output back
     ds0 = dss[0]
-    host_in = {k: torch.from_numpy(np.ascontiguousarray(a)) for k, a in (
-        ("q", step.q), ("k_new", step.k_new), ("v_new", step.v_new),
-        ("slot_mapping", ds0.plan.slot_mapping), ("block_tables", ds0.plan.block_tables),
-        ("seq_lens", ds0.plan.seq_lens), ("query_start_loc", ds0.plan.query_start_loc))}
-    host_in = {k: v.pin_memory() for k, v in host_in.items()}
+    host_ins = [d.host_inputs() for d in dss]
     host_out = torch.empty(ds0.out.shape, dtype=torch.int16).pin_memory()
-    dev_views = [{"q": d.q.view(torch.int16), "k_new": d.k_new.view(torch.int16),
-                  "v_new": d.v_new.view(torch.int16), "slot_mapping": d.slot_mapping,
-                  "block_tables": d.block_tables, "seq_lens": d.seq_lens,
-                  "query_start_loc": d.query_start_loc} for d in dss]
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    h2d = host_ins[0].numel()
     d2h = host_out.numel() * host_out.element_size()
 
-    def e2e_step(i):
-        d, view = dss[i % copies], dev_views[i % copies]
-        for k, hv in host_in.items():
-            view[k].copy_(hv.view(view[k].dtype), non_blocking=True)
-        d.run()
-        host_out.copy_(d.out.view(torch.int16), non_blocking=True)
-
     def e2e_graph(r):
-        d, view = dss[r], dev_views[r]
+        d, hin = dss[r], host_ins[r]
 
         def copies_in():
-            for k, hv in host_in.items():
-                view[k].copy_(hv.view(view[k].dtype), non_blocking=True)
+            d.inputs.copy_(hin, non_blocking=True)
 
         def copy_out():
             host_out.copy_(d.out.view(torch.int16), non_blocking=True)
@@ -454,7 +439,7 @@ def bench_ours(args) -> None:
     barrier(world)
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_value = bytes_all / (e2e_ms / 1e3) / 1e9
-    del dss, host_in, dev_views, ds0, step_graphs, attn_graphs, e2e_graphs
+    del dss, host_ins, ds0, step_graphs, attn_graphs, e2e_graphs
     torch.cuda.empty_cache()
     mixed = None if args.no_mixed else bench_mixed(args, dev, stream, world, clocks)
     clk = clocks.stop() if clocks else None

@@ -19,6 +19,10 @@ from .block_pool import plan_step
 from .inputs import StepInputs
 
 
+_TORCH_DTYPE = {np.dtype(np.uint16): torch.bfloat16, np.dtype(np.float32): torch.float32,
+                np.dtype(np.int32): torch.int32, np.dtype(np.int64): torch.int64}
+
+
 def to_torch(a: np.ndarray, device) -> torch.Tensor:
     """numpy array (float32, or uint16 holding bf16 bits, or ints) -> torch tensor."""
     t = torch.from_numpy(np.ascontiguousarray(a))
@@ -51,17 +55,36 @@ class DeviceStep:
             lib.reshape_and_cache(to_torch(step.k_ctx[s:e], device),
                                   to_torch(step.v_ctx[s:e], device), self.k_cache, self.v_cache,
                                   to_torch(plan.ctx_slot_mapping[s:e], device))
-        self.q = to_torch(step.q, device)
-        self.k_new = to_torch(step.k_new, device)
-        self.v_new = to_torch(step.v_new, device)
-        self.block_tables = to_torch(plan.block_tables, device)
-        self.seq_lens = to_torch(plan.seq_lens, device)
-        self.query_start_loc = to_torch(plan.query_start_loc, device)
-        self.slot_mapping = to_torch(plan.slot_mapping, device)
+        # the step's inputs live in one contiguous device buffer (each 256-byte
+        # aligned), so that a caller bringing them from the host needs one copy
+        self._input_arrays = [("q", step.q), ("k_new", step.k_new), ("v_new", step.v_new),
+                              ("slot_mapping", plan.slot_mapping),
+                              ("block_tables", plan.block_tables),
+                              ("seq_lens", plan.seq_lens),
+                              ("query_start_loc", plan.query_start_loc)]
+        self._layout, total = [], 0
+        for name, a in self._input_arrays:
+            a = np.ascontiguousarray(a)
+            self._layout.append((name, total, a.nbytes, a.dtype, a.shape))
+            total += (a.nbytes + 255) // 256 * 256
+        self.inputs = torch.empty(total, dtype=torch.uint8, device=device)
+        for (name, off, nbytes, dt, shape), (_, a) in zip(self._layout, self._input_arrays):
+            view = self.inputs[off:off + nbytes].view(_TORCH_DTYPE[np.dtype(dt)]).view(shape)
+            view.copy_(to_torch(np.ascontiguousarray(a), "cpu"))
+            setattr(self, name, view)
         self.out = torch.empty_like(self.q)
         self.workspace = lib.new_workspace(step.num_seqs, step.num_q_heads, step.num_kv_heads,
                                            step.head_dim, max(1, plan.max_seq_len), device)
         torch.cuda.synchronize()
+
+    def host_inputs(self) -> torch.Tensor:
+        """A pinned host copy of ``inputs`` (same layout): one H2D copy of it
+        into ``inputs`` gives the step all of its inputs."""
+        host = torch.zeros(self.inputs.numel(), dtype=torch.uint8).pin_memory()
+        for (name, off, nbytes, dt, shape), (_, a) in zip(self._layout, self._input_arrays):
+            host[off:off + nbytes].copy_(
+                torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)))
+        return host
 
     def write_new_tokens(self, stream=None) -> None:
         lib.reshape_and_cache(self.k_new, self.v_new, self.k_cache, self.v_cache,

@@ -373,3 +373,22 @@ def test_decode_partition_edge_steps(case, hints):
                          seq_lens=np.concatenate([step.seq_lens, [700]]),
                          query_lens=np.concatenate([step.query_lens, [300]]), seed=7)
     run_and_check(step, host_hints=hints)
+
+
+def test_packed_inputs_one_host_copy():
+    """A step's inputs are one device buffer: one H2D copy of host_inputs()
+    restores all of them, and the step then gives the same bytes."""
+    from paged_kv_cache_469_b200.step import DeviceStep
+    step = random_step(101, dtype="bf16", num_q_heads=32, num_kv_heads=4, head_dim=64,
+                       num_seqs=6, max_ctx=500, max_q=2)
+    ds = DeviceStep(step)
+    ds.run_fused()
+    torch.cuda.synchronize()
+    ref = _bits(ds.out).copy()
+    host = ds.host_inputs()
+    ds.inputs.zero_()
+    ds.inputs.copy_(host, non_blocking=True)
+    ds.out.zero_()
+    ds.run_fused()
+    torch.cuda.synchronize()
+    assert _bits(ds.out).tobytes() == ref.tobytes()
