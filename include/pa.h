@@ -18,11 +18,20 @@
  * Conventions of every call:
  *   - Every tensor pointer is DEVICE memory owned by the caller, contiguous,
  *     row-major, 16-byte aligned.  The library allocates nothing and keeps no
- *     state between calls; the caller's workspace holds all scratch.
+ *     data between calls; the caller's workspace holds all scratch.  (It does
+ *     remember, per device, the kernel attributes it has already set.)
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
- *     legacy default stream).  Argument checks run on the host before any
- *     launch and return PA_ERR_INVALID / PA_ERR_UNSUPPORTED with nothing
- *     launched; PA_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *     legacy default stream) and keeps stream order: each kernel is launched
+ *     as a programmatic dependent of the work before it, so its launch may
+ *     overlap that work's tail, but it reads and writes nothing until that
+ *     work has completed.  Argument checks run on the host before any launch
+ *     and return PA_ERR_INVALID / PA_ERR_UNSUPPORTED with nothing launched;
+ *     PA_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *   - Calls can be captured in a CUDA graph.  A capture records the launch
+ *     plan of that call: with the optional host copies of seq_lens and
+ *     query_start_loc, that plan follows them (kernel choice, split-K
+ *     partition length, the prefill work list), so a replay needs device
+ *     arrays that still hold those values.
  *   - Nothing traps on the device.  Slots or block ids outside the pool are
  *     never dereferenced (see each call).
  *   - dtype is the element type of q, k, v, the caches and out alike.
@@ -140,8 +149,11 @@ int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_s
  *                  num_kv_heads, head_dim, max_seq_len) bytes, zeroed once by
  *                  pa_workspace_init; one workspace serves one call at a time
  *   seq_lens_host, query_start_loc_host  optional (NULL) host copies of the
- *                  two device arrays: when given, the call checks them and
- *                  launches only the kernels the step needs
+ *                  two device arrays, equal to them: when given, the call
+ *                  checks them, launches only the kernels the step needs,
+ *                  sizes the split-K partitions from the step's total keys,
+ *                  and (up to 1024 prefill work items) passes the prefill work
+ *                  list with the launch instead of building it on the GPU
  *
  * Decode-class sequences (q_len * num_q_heads / num_kv_heads <= 16 query
  * rows per kv-head) run the split-K bandwidth-bound kernel; longer prefill
