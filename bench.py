@@ -278,11 +278,11 @@ def timed_loop(fns, stream, steps: int) -> float:
 
 def prefill_flops(step) -> int:
     """Flops of the unmasked (query, key) pairs of the prefill-class sequences
-    (q_len * group > 16): 4 * D * Hq per pair (Q.K^T and P.V)."""
+    (q_len * group > 64): 4 * D * Hq per pair (Q.K^T and P.V)."""
     g = step.num_q_heads // step.num_kv_heads
     pairs = 0
     for ql, L in zip(step.query_lens.tolist(), step.seq_lens.tolist()):
-        if ql * g > 16:
+        if ql * g > 64:
             pairs += ql * (L - ql) + ql * (ql + 1) // 2
     return 4 * step.head_dim * step.num_q_heads * pairs
 
@@ -308,7 +308,7 @@ def bench_mixed(args, dev, stream, world, clocks):
     tokens = sum_over_ranks(step.num_tokens, world)
     g = step.num_q_heads // step.num_kv_heads
     kv_dec = int(sum(L for L, q in zip(step.seq_lens.tolist(), step.query_lens.tolist())
-                     if q * g <= 16)) * 2 * step.num_kv_heads * step.head_dim * 2
+                     if q * g <= 64)) * 2 * step.num_kv_heads * step.head_dim * 2
     copies = len(dss)
     del dss, graphs
     torch.cuda.empty_cache()

@@ -155,9 +155,10 @@ int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_s
  *                  and (up to 1024 prefill work items) passes the prefill work
  *                  list with the launch instead of building it on the GPU
  *
- * Decode-class sequences (q_len * num_q_heads / num_kv_heads <= 16 query
- * rows per kv-head) run the split-K bandwidth-bound kernel; longer prefill
- * chunks run the tensor-core kernel.  fp32 steps run a CUDA-core kernel.
+ * Decode-class sequences (q_len * num_q_heads / num_kv_heads <= 64 query
+ * rows per kv-head: single-token decodes and the few-token queries of
+ * speculative verification) run the split-K bandwidth-bound kernel, 16 rows
+ * per CTA; longer prefill chunks run the tensor-core kernel.  fp32 steps run a CUDA-core kernel.
  * Supported: head_dim in {64, 128}; block_size 16; num_q_heads a multiple of
  * num_kv_heads with at most 16 q-heads per kv-head; dtype f32 or bf16;
  * max_seq_len up to at least 1.5M tokens (a longer bound than the split-K

@@ -129,7 +129,8 @@ decode_splitk_kernel(const AttnParams p) {
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = lane >> 2, q4 = lane & 3;
-  const int s = blockIdx.z, kvh = blockIdx.y, part = blockIdx.x;
+  const int s = blockIdx.z, part = blockIdx.x;
+  const int kvh = blockIdx.y / p.row_groups, rg = blockIdx.y % p.row_groups;
 
   // Launched as a programmatic dependent: the CTA may be resident before the
   // preceding kernel on the stream (typically the cache write) has finished;
@@ -142,13 +143,19 @@ decode_splitk_kernel(const AttnParams p) {
   const int ql = p.query_start_loc[s + 1] - q0;
   const int L = p.seq_lens[s];
   const int G = p.group;
-  const int rows = ql * G;
-  if (ql <= 0 || ql > L || rows > (kRows16 ? 16 : 8)) return;
+  // this CTA's query rows of the (sequence, kv-head): global rows row0 ..
+  // row0 + rows - 1, global row i being token i / G, q-head kvh * G + i % G
+  const int rows_all = ql * G;
+  const int row0 = kDecodeRows * rg;
+  const int rows = min(kDecodeRows, rows_all - row0);
+  if (ql <= 0 || ql > L || rows_all > kDecodeMaxRows || rows <= 0 ||
+      rows > (kRows16 ? 16 : 8))
+    return;
   const int P = p.part_tokens;
   const int nparts = (L + P - 1) / P;
   // a sequence longer than the bounds the workspace was sized for is left
   // unwritten rather than overrunning the workspace or its block-table row
-  if (part >= nparts || nparts > p.max_parts || L > p.max_seq_len ||
+  if (part >= nparts || nparts * p.row_groups > p.max_parts || L > p.max_seq_len ||
       (L + kBlockSize - 1) / kBlockSize > p.max_blocks_per_seq)
     return;
   // nparts partitions of equal whole blocks (the last may be shorter; with
@@ -210,9 +217,9 @@ decode_splitk_kernel(const AttnParams p) {
   uint32_t qa[NC][2], qb[NC][2];
   {
     const bool va = r < rows, vb = kRows16 && (r + 8) < rows;
-    const int64_t ra = va ? ((int64_t)(q0 + r / G) * p.num_q_heads + kvh * G + r % G) * D : 0;
-    const int64_t rb =
-        vb ? ((int64_t)(q0 + (r + 8) / G) * p.num_q_heads + kvh * G + (r + 8) % G) * D : 0;
+    const int ga = row0 + r, gb = row0 + r + 8;
+    const int64_t ra = va ? ((int64_t)(q0 + ga / G) * p.num_q_heads + kvh * G + ga % G) * D : 0;
+    const int64_t rb = vb ? ((int64_t)(q0 + gb / G) * p.num_q_heads + kvh * G + gb % G) * D : 0;
 #pragma unroll
     for (int jp = 0; jp < NJ; ++jp) {
       uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
@@ -223,8 +230,8 @@ decode_splitk_kernel(const AttnParams p) {
     }
   }
   // causal limit of rows r and r+8: query j sees keys <= L - ql + j
-  const int lim_a = L - ql + min(r, rows - 1) / G;
-  const int lim_b = L - ql + min(r + 8, rows - 1) / G;
+  const int lim_a = L - ql + (row0 + min(r, rows - 1)) / G;
+  const int lim_b = L - ql + (row0 + min(r + 8, rows - 1)) / G;
   const int first_masked = L - ql + 1;  // keys at or beyond this may be masked for some row
 
   const char* kc = (const char*)p.k_cache;
@@ -416,11 +423,12 @@ decode_splitk_kernel(const AttnParams p) {
       Os += sh_o[w][row][d] * f;
     }
     if (direct) {
-      const int tok = q0 + row / G, head = kvh * G + row % G;
+      const int tok = q0 + (row0 + row) / G, head = kvh * G + (row0 + row) % G;
       out[((int64_t)tok * p.num_q_heads + head) * D + d] =
           __float2bfloat16_rn(Ls > 0.f ? Os / Ls : 0.f);
     } else {
-      const int64_t slot = ((int64_t)unit * p.max_parts + part) * kDecodeRows + row;
+      const int64_t slot =
+          ((int64_t)unit * p.max_parts + part * p.row_groups + rg) * kDecodeRows + row;
       p.ws_o[slot * D + d] = Os;
       if (d == 0) { p.ws_ml[slot * 2] = M; p.ws_ml[slot * 2 + 1] = Ls; }
     }
@@ -431,7 +439,7 @@ decode_splitk_kernel(const AttnParams p) {
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    const int prev = atomicAdd(p.ws_counter + unit, 1);
+    const int prev = atomicAdd(p.ws_counter + unit * kDecodeRowGroups + rg, 1);
     sh_last = (prev == nparts - 1);
     if (sh_last) __threadfence();
   }
@@ -443,11 +451,13 @@ decode_splitk_kernel(const AttnParams p) {
   float* sh_pm = reinterpret_cast<float*>(smem);  // [nparts][kDecodeRows] max, then weight
   float* sh_pl = sh_pm + nparts * kDecodeRows;    // [nparts][kDecodeRows] sum
   float* sh_inv = sh_pl + nparts * kDecodeRows;   // [kDecodeRows] 1 / merged sum
-  const int64_t unit_slot = (int64_t)unit * p.max_parts * kDecodeRows;
+  // partition q of this row group is partial slot q * row_groups + rg of the unit
+  const int64_t unit_slot = ((int64_t)unit * p.max_parts + rg) * kDecodeRows;
+  const int slot_step = p.row_groups * kDecodeRows;
   for (int i = threadIdx.x; i < nparts * rows; i += blockDim.x) {
     const int q = i / rows, row = i % rows;
     const float2 ml =
-        __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + unit_slot + q * kDecodeRows + row);
+        __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + unit_slot + q * slot_step + row);
     sh_pm[q * kDecodeRows + row] = ml.x;
     sh_pl[q * kDecodeRows + row] = ml.y;
   }
@@ -473,18 +483,18 @@ decode_splitk_kernel(const AttnParams p) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int q = 0; q < nparts; ++q) {
-      const float4 v = __ldcg(po + (unit_slot + q * kDecodeRows + row) * D4 + d4);
+      const float4 v = __ldcg(po + (unit_slot + q * slot_step + row) * D4 + d4);
       const float f = sh_pm[q * kDecodeRows + row];
       acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
     }
     const float inv = sh_inv[row];
-    const int tok = q0 + row / G, head = kvh * G + row % G;
+    const int tok = q0 + (row0 + row) / G, head = kvh * G + (row0 + row) % G;
     uint2 pk;
     pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
     pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
     *reinterpret_cast<uint2*>(out + ((int64_t)tok * p.num_q_heads + head) * D + 4 * d4) = pk;
   }
-  if (threadIdx.x == 0) p.ws_counter[unit] = 0;  // ready for the next call
+  if (threadIdx.x == 0) p.ws_counter[unit * kDecodeRowGroups + rg] = 0;  // ready for the next call
 }
 
 template <int D, bool kRows16, int kStages, bool kWriteCache>
@@ -502,7 +512,7 @@ cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   const int parts = (p.max_seq_len + p.part_tokens - 1) / p.part_tokens;  // <= p.max_parts
-  cfg.gridDim = dim3(parts > 0 ? parts : 1, p.num_kv_heads, p.num_seqs);
+  cfg.gridDim = dim3(parts > 0 ? parts : 1, p.num_kv_heads * p.row_groups, p.num_seqs);
   cfg.blockDim = dim3(kWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -549,7 +559,8 @@ int decode_wave_ctas(int head_dim, int rows) {
 cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
                                  cudaStream_t stream) {
   if (p.num_seqs == 0) return cudaSuccess;
-  const int max_rows = min(max_query_len * p.group, kDecodeRows);
+  const int max_rows = min(p.decode_rows > 0 ? p.decode_rows : max_query_len * p.group,
+                           kDecodeRows);
   const bool rows16 = max_rows > 8;
   cudaError_t e;
   constexpr int s64 = PA_DECODE_STAGES_D64, s128 = PA_DECODE_STAGES_D128;

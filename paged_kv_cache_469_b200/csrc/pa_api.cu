@@ -45,7 +45,9 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads
                                  int max_seq_len) {
   WorkspaceLayout w{};
   w.part_tokens = part_tokens_floor(max_seq_len);
-  w.max_parts = max(1, (max_seq_len + w.part_tokens - 1) / w.part_tokens);
+  // a slot per (partition, row group): at least one partition for each of the
+  // row groups a multi-token decode may need
+  w.max_parts = max(kDecodeRowGroups, (max_seq_len + w.part_tokens - 1) / w.part_tokens);
   // prefill items: at most ceil(q_len / 128) <= ceil(max_seq_len / 128) per sequence and q-head
   const long items = (long)num_seqs * ((max_seq_len + kPrefillQTile - 1) / kPrefillQTile) *
                      num_q_heads;
@@ -54,7 +56,8 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads
   const size_t slots = units * w.max_parts * kDecodeRows;
   w.status_off = 0;
   w.counter_off = 256;
-  w.o_off = align_up(w.counter_off + units * sizeof(int), 256);
+  // one arrival counter per (sequence, kv-head, row group)
+  w.o_off = align_up(w.counter_off + units * kDecodeRowGroups * sizeof(int), 256);
   w.ml_off = align_up(w.o_off + slots * head_dim * sizeof(float), 256);
   w.items_off = align_up(w.ml_off + slots * 2 * sizeof(float), 256);
   w.total = align_up(w.items_off + (size_t)(w.max_items + 1) * 16, 256);
@@ -166,26 +169,29 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
   bool any_decode = true, any_prefill = true;
   int prefill_items = -1;  // unknown without the host copies
   long decode_keys = -1;   // sum of the decode-class sequences' lengths, when known
+  int decode_rows = min(max_query_len * group, kDecodeMaxRows);  // most rows of one of them
   if (seq_lens_host && query_start_loc_host) {
     if (query_start_loc_host[0] != 0 || query_start_loc_host[num_seqs] != num_tokens)
       return PA_ERR_INVALID;
     any_decode = any_prefill = false;
     prefill_items = 0;
     decode_keys = 0;
+    decode_rows = 0;
     for (int s = 0; s < num_seqs; ++s) {
       const int ql = query_start_loc_host[s + 1] - query_start_loc_host[s];
       const int L = seq_lens_host[s];
       if (ql < 0 || ql > L || L > max_seq_len || ql > max_query_len) return PA_ERR_INVALID;
       if (ql == 0) continue;
-      if (ql * group <= kDecodeRows) {
+      if (ql * group <= kDecodeMaxRows) {
         any_decode = true;
         decode_keys += L;
+        decode_rows = max(decode_rows, ql * group);
       } else {
         any_prefill = true;
         prefill_items += (ql + kPrefillQTile - 1) / kPrefillQTile * num_q_heads;
       }
     }
-  } else if (max_query_len * group <= kDecodeRows) {
+  } else if (max_query_len * group <= kDecodeMaxRows) {
     any_prefill = false;
   }
 
@@ -204,10 +210,17 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
   p.max_seq_len = max_seq_len;
   p.max_parts = w.max_parts;  // the workspace's partitions per (sequence, kv-head)
   {
+    p.row_groups = max(1, (decode_rows + kDecodeRows - 1) / kDecodeRows);
+    p.decode_rows = decode_rows;
+    const int rows = max(1, min(decode_rows, kDecodeRows));  // per CTA
     const long keys = decode_keys >= 0 ? decode_keys : (long)num_seqs * (max_seq_len / 2 + 1);
-    const int rows = min(max_query_len * group, kDecodeRows);
-    p.part_tokens = part_tokens_for_step(keys * num_kv_heads,
-                                         decode_wave_ctas(head_dim, rows), w.part_tokens);
+    int part = part_tokens_for_step(keys * num_kv_heads * p.row_groups,
+                                    decode_wave_ctas(head_dim, rows), w.part_tokens);
+    // the slots of one (sequence, kv-head) hold every (partition, row group)
+    const int parts_cap = max(1, w.max_parts / p.row_groups);
+    const long need = ((long)max_seq_len + parts_cap - 1) / parts_cap;
+    if (need > part) part = (int)((need + kBlockSize - 1) / kBlockSize * kBlockSize);
+    p.part_tokens = part;
   }
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;

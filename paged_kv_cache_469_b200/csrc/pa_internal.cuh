@@ -32,6 +32,11 @@ inline cudaError_t raise_smem_limit(Kernel kernel, int bytes, std::atomic<int> (
 
 constexpr int kBlockSize = 16;       // tokens per cache block (the pages' default)
 constexpr int kDecodeRows = 16;      // query rows per kv-head one decode CTA holds (MMA M)
+// A decode-class sequence has at most kDecodeMaxRows query rows per kv-head
+// (q_len * q-heads per kv-head); they are split into 16-row groups, one CTA
+// each.  Longer queries are prefill chunks.
+constexpr int kDecodeRowGroups = 4;
+constexpr int kDecodeMaxRows = kDecodeRows * kDecodeRowGroups;
 // split-K partitions per sequence the decode kernel can merge (its shared
 // memory holds each partition's per-row max and sum): 1536 partitions of at
 // least 1024 keys, i.e. sequences of at least 1.5M tokens
@@ -69,7 +74,10 @@ struct AttnParams {
   const int64_t* slot_mapping;
   int part_tokens;   // keys per partition at most (multiple of 16); a sequence is cut
                      // into ceil(L / part_tokens) partitions of equal whole blocks
-  int max_parts;     // partitions the workspace holds per (sequence, kv-head)
+  int max_parts;     // partial slots the workspace holds per (sequence, kv-head): one per
+                     // (partition, row group), partition-major
+  int row_groups;    // 16-row groups per (sequence, kv-head) in this launch (1..4)
+  int decode_rows;   // most query rows of one decode-class (sequence, kv-head)
   float* ws_o;       // [num_seqs*Hkv][max_parts][16][D] unnormalised partial outputs
   float* ws_ml;      // [num_seqs*Hkv][max_parts][16][2] running max (log2 units), sum
   int* ws_counter;   // [num_seqs*Hkv] arrival counters, zero between calls

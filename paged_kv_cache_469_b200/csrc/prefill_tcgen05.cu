@@ -719,7 +719,7 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
 
 // --------------------------------------------------------------- work list
 
-// One CTA: list the prefill items of every sequence with q_len * group > 16,
+// One CTA: list the prefill items of every sequence with q_len * group > 64,
 // heaviest (most key tiles) first (a counting sort on the tile count), and
 // store the count in ws_items[0].x.  An item pairs two q-heads of one kv-head
 // (pair_heads: the group is even) or two consecutive query tiles of one
@@ -744,7 +744,7 @@ prefill_plan_kernel(const AttnParams p, int max_tiles, int pair_heads) {
   // pass 1: histogram of items by tile count
   for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
     const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
-    if (ql * p.group <= kDecodeRows || ql > L) continue;
+    if (ql * p.group <= kDecodeMaxRows || ql > L) continue;
     const int nq = (ql + QT - 1) / QT;
     const int ni = pair_heads ? nq : (nq + 1) / 2;
     for (int i = 0; i < ni; ++i) {
@@ -768,7 +768,7 @@ prefill_plan_kernel(const AttnParams p, int max_tiles, int pair_heads) {
   // pass 2: scatter
   for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
     const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
-    if (ql * p.group <= kDecodeRows || ql > L) continue;
+    if (ql * p.group <= kDecodeMaxRows || ql > L) continue;
     const int nq = (ql + QT - 1) / QT;
     const int ni = pair_heads ? nq : (nq + 1) / 2;
     for (int i = ni - 1; i >= 0; --i) {
@@ -837,7 +837,7 @@ bool host_work_list(PrefillWork* work, const AttnParams& p, const int32_t* seq_l
     for (int s = 0; s < p.num_seqs; ++s) {
       const int ql = query_start_loc_host[s + 1] - query_start_loc_host[s];
       const int L = seq_lens_host[s];
-      if (ql * p.group <= kDecodeRows || ql > L) continue;
+      if (ql * p.group <= kDecodeMaxRows || ql > L) continue;
       const int nq = (ql + QT - 1) / QT;
       const int ni = pair_heads ? nq : (nq + 1) / 2;
       for (int i = 0; i < ni; ++i) {

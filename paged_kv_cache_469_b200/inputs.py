@@ -209,7 +209,7 @@ def workload(name: str, *, with_values: bool = True) -> StepInputs:
     raise KeyError(name)
 
 
-def prefill_part(step: StepInputs, decode_rows: int = 16) -> StepInputs:
+def prefill_part(step: StepInputs, decode_rows: int = 64) -> StepInputs:
     """A step of the same shape holding only ``step``'s prefill-class sequences
     (q_len * group > ``decode_rows``), with the same lengths, fresh draws from
     the same seed and a pool just large enough for them."""

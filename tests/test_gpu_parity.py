@@ -65,7 +65,7 @@ def run_and_check(step, *, full=True, rows=None, check_cache=True, host_hints=Tr
                                           num_threads=NTHREADS)
         assert_close(got[tok, head], ref, step.dtype, step.name + " (sampled rows)")
     # split-K counters (after the 256-byte status block) are back at zero
-    n = step.num_seqs * step.num_kv_heads * 4
+    n = step.num_seqs * step.num_kv_heads * 4 * 4  # four row groups
     assert int(ds.workspace[256:256 + n].count_nonzero()) == 0
     return ds, st
 
@@ -295,7 +295,7 @@ def _fused_check(step, host_hints=True, d_dtype="bf16"):
     assert _bits(ds.v_cache).tobytes() == st["v_cache"].tobytes(), "v_cache differs"
     assert_close(ds.out_f64(), oracle_outputs(step, st, num_threads=NTHREADS), step.dtype,
                  step.name + " (one call)")
-    n = step.num_seqs * step.num_kv_heads * 4
+    n = step.num_seqs * step.num_kv_heads * 4 * 4  # four row groups
     assert int(ds.workspace[256:256 + n].count_nonzero()) == 0
     return ds
 
@@ -392,3 +392,31 @@ def test_packed_inputs_one_host_copy():
     ds.run_fused()
     torch.cuda.synchronize()
     assert _bits(ds.out).tobytes() == ref.tobytes()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hq,hkv,ql", [(32, 4, 3), (32, 4, 8), (32, 8, 5), (32, 8, 16),
+                                       (16, 1, 3), (8, 8, 40), (32, 8, 17)])
+@pytest.mark.parametrize("hints", [True, False])
+def test_multi_token_decode_row_groups(d, hq, hkv, ql, hints):
+    """Queries of 17..64 rows per kv-head (q_len * group) stay on the split-K
+    decode kernel as up to four 16-row groups (one CTA each, each with its own
+    partials and merge), mixed with one-token decodes and, for (32, 8, 17),
+    with a prefill-class neighbour (68 rows)."""
+    lens = [5000, 37, 300, 16, ql, 1200]
+    qls = [ql, 1, ql, 1, ql, min(ql, 1200)]
+    step = make_step(name="mtd_rg", dtype="bf16", num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+                     num_blocks=int(np.sum((np.array(lens) + 15) // 16)) + 30, seq_lens=lens,
+                     query_lens=qls, seed=11 + ql)
+    run_and_check(step, host_hints=hints)
+
+
+@pytest.mark.parametrize("ql", [3, 8])
+def test_write_cache_call_row_groups(ql):
+    """The one-call path on multi-token decodes: every row group of a partition
+    writes the same new rows and reads them back."""
+    lens = np.array([2100, 700, 33, ql])
+    step = make_step(name="fused_rg", dtype="bf16", num_q_heads=32, num_kv_heads=4, head_dim=64,
+                     num_blocks=int(np.sum((lens + 15) // 16)) + 20, seq_lens=lens,
+                     query_lens=np.full(4, ql), seed=23 + ql)
+    _fused_check(step)
