@@ -41,7 +41,7 @@ MAX_COPIES = 8
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode_splitk_kernel<64,false,4,4,false>
 # launch on this workload, from an ncu --set full capture of that launch; set
 # to None whenever that kernel changes, until it is captured again
-DECODE_TRAFFIC_BYTES = 68_941_312 + 962_816
+DECODE_TRAFFIC_BYTES = 68_948_736 + 1_102_080
 
 
 def kv_bytes(step, seqs=None) -> int:
