@@ -5,13 +5,15 @@
 // bandwidth; section "PagedAttentionの仕組み": the keys are read block by
 // block through the sequence's block table.
 //
-// Work split.  One CTA (kWarps warps) per (partition of part_tokens keys,
-// kv-head, sequence); the hardware hands CTAs to SMs as they free up, which
-// balances the load even though SMs do not all get the same share of memory
-// bandwidth.  All q-heads of the kv-head (and, for a short multi-token
-// decode, all its query tokens) form the rows of one 16-row MMA tile, so every
-// K/V byte is read from HBM once per kv-head.  Warp w of the CTA takes blocks
-// w, w+kWarps, ... of the partition.
+// Work split.  One CTA (kWarps warps) per (partition, kv-head and row group,
+// sequence): a sequence of L keys is cut into ceil(L / part_tokens)
+// partitions of equal whole blocks; the hardware hands CTAs to SMs as they
+// free up.  The query rows of a (sequence, kv-head) -- all q-heads of the
+// kv-head times its query tokens, up to 64 -- are cut into 16-row groups, each
+// the rows of one 16-row MMA tile in its own CTA; a single-token decode with
+// up to 16 q-heads per kv-head is one group, so every K/V byte is read from
+// HBM once per kv-head.  Warp w of the CTA takes blocks w, w+kWarps, ... of
+// the partition.
 //
 // Staging.  Each warp streams its blocks through a private ring of kStages
 // shared-memory slots (one (block, kv-head) K tile + V tile per slot) with
@@ -36,7 +38,9 @@
 //
 // The kernel is launched as a programmatic dependent of whatever precedes it
 // on the stream (typically the cache write), so its launch overlaps that
-// kernel's tail; it reads nothing before griddepcontrol.wait.
+// kernel's tail; it reads nothing before griddepcontrol.wait.  In the
+// one-call form (kWriteCache) it first stores the step's new K/V rows that
+// fall in its own partition into their cache slots, then reads them back.
 #include <math.h>
 
 #include "pa_internal.cuh"

@@ -7,28 +7,33 @@
 // through the sequence's block table and a causal, position-based mask keeps
 // each query on its own sequence's earlier tokens.
 //
-// Work item = (sequence, 128-query tile, q-head).  A persistent CTA walks its
-// items; per item it streams the sequence's keys in 128-key tiles:
+// Work item = (sequence, 128-query tile, two q-heads of one kv-head), or two
+// consecutive 128-query tiles of one q-head when the group size is odd: two
+// 128-row halves that read the same keys.  A persistent CTA (one per SM)
+// walks its items, heaviest first; per item it streams the sequence's keys in
+// 128-key tiles:
 //
-//   warps 8, 10 TMA producers (warp 8: the two Q tiles once per item, then K
-//               tiles; warp 10: V tiles), each tile eight 16-token cache
-//               blocks (one 16 x 64 box per block and 64-wide slice of D,
-//               128-byte swizzled, straight from the pool through the block
-//               table)
-//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (tcgen05.mma,
-//               M=128, N=128, K=16 steps), then O += P V into TMEM
-//   warps 2..5  softmax: one query row per thread; S from TMEM (tcgen05.ld),
-//               causal mask, online softmax in fp32 (exp2, the running max is
-//               only moved when it grows by more than 2^8, so O is rarely
-//               rescaled), P as bf16 into shared memory (double-buffered) for
-//               the second MMA;
-//               at the end of the item O / l from TMEM to global memory
+//   warp 8      TMA: the two Q tiles once per item, then every K tile -- eight
+//               16-token cache blocks, one 16 x 64 box per block and 64-wide
+//               slice of D, 128-byte swizzled, straight from the pool through
+//               the block table
+//   warp 10     TMA: every V tile, the same way
+//   warp 9      MMA issuer (one thread): S_h = Q_h K^T into TMEM (tcgen05.mma,
+//               M=128, N=128, K=16 steps, both operands in shared memory), and
+//               O_h += P_h V with P_h read from TMEM
+//   warps 0..3, 4..7  softmax of half 0 / half 1, one query row per thread:
+//               S from TMEM (tcgen05.ld), causal mask, online softmax in fp32
+//               (exp2; the running max moves only when it grows by more than
+//               2^8, so O is rarely rescaled), P as bf16 written back over S
+//               in TMEM (tcgen05.st); at the end of the item O / l to global
+//               memory
 //
-// S is double-buffered in TMEM so that Q K^T of tile j+1 overlaps the softmax
-// of tile j.  The last, partly filled cache block of a sequence is loaded at a
-// negative row offset so that its unwritten slots arrive as TMA zero fill
-// (never uninitialised cache memory); blocks past the sequence, or block ids
-// outside the pool, are loaded from beyond the tensor's extent (zeros).
+// The MMA warp issues P.V of tile g-1 before Q K^T of tile g for each half, so
+// the tensor pipe works on one half while the softmax of the other runs.  The
+// last, partly filled cache block of a sequence is loaded at a negative row
+// offset so that its unwritten slots arrive as TMA zero fill (never
+// uninitialised cache memory); blocks past the sequence, or block ids outside
+// the pool, are loaded from beyond the tensor's extent (zeros).
 //
 // Every mbarrier wait is bounded by a time limit; a wait that runs out sets a
 // status bit in the workspace and the CTA winds down instead of hanging.
