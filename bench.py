@@ -214,6 +214,17 @@ def oracle_sample(step, target_s: float, threads: int):
     return kv_bytes(step, np.arange(n)) * passes / total / 1e9, n, total, run, passes
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def bench_reference(args) -> None:
     """The CPU oracle as the reference arm: each step is one pass over a bounded
     sample of the workload, on the host cores."""
@@ -462,9 +473,14 @@ def bench_ours(args) -> None:
     if world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
         gbs, n, dt, _, passes = oracle_sample(step, target_s=10.0, threads=threads)
+        gbs1, n1, dt1, _, passes1 = oracle_sample(step, target_s=4.0, threads=1)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"first {n} of {step.num_seqs} sequences (all q-heads), {passes} "
-                         f"passes, {dt:.1f} s"}
+                         f"passes, {dt:.1f} s",
+               "single_thread": {"value": round(gbs1, 4), "unit": "GB/s",
+                                 "sample": f"first {n1} sequences, {passes1} passes, "
+                                           f"{dt1:.1f} s"},
+               "cpu_model": cpu_model()}
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
