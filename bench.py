@@ -355,6 +355,98 @@ def bench_mixed(args, dev, stream, world, clocks):
                                          "host copies of the step's lengths)")}}
 
 
+def bench_planner(args, dev, stream) -> dict:
+    """The on-GPU step planner (pa_plan_step) on the decode workload's step:
+    device time per call, against the host path it replaces (BlockPool,
+    numpy slot mapping and prefix sum, pinned copies to the device)."""
+    import numpy as np
+    import torch
+    from paged_kv_cache_469_b200 import block_pool, lib
+    from paged_kv_cache_469_b200.inputs import workload
+    step = workload(WORKLOAD, with_values=False)
+    S = step.num_seqs
+    ql = step.query_lens.astype(np.int32)
+    nc = (step.seq_lens - step.query_lens).astype(np.int32)
+    mb = max(1, -(-int(step.seq_lens.max()) // 16))
+
+    def host_pool():
+        pool = block_pool.BlockPool(step.free_queue)
+        for s in range(S):
+            pool.allocate_slots(s, int(nc[s]))
+        return pool
+
+    pool = host_pool()
+    head0 = len(step.free_queue) - len(pool.free_block_queue)
+    tables0 = pool.block_table(range(S), mb)
+    for s in range(S):
+        pool.allocate_slots(s, int(nc[s] + ql[s]))
+    tables1 = pool.block_table(range(S), mb)
+    slots1 = block_pool.slot_mapping(tables1, nc, ql)
+    qsl1 = block_pool.query_start_loc(ql)
+    per_call = len(step.free_queue) - len(pool.free_block_queue) - head0
+
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    fq, tables, nc_t, ql_t = t(step.free_queue), t(tables0), t(nc), t(ql)
+    state = lib.new_planner_state(head0, device=dev)
+    seq_lens = torch.empty(S, dtype=torch.int32, device=dev)
+    qsl = torch.empty(S + 1, dtype=torch.int32, device=dev)
+    slots = torch.empty(int(ql.sum()), dtype=torch.int64, device=dev)
+
+    def call():
+        lib.plan_step(fq, state, nc_t, ql_t, tables, seq_lens, qsl, slots, stream=stream)
+
+    call()
+    torch.cuda.synchronize(dev)
+    # both product paths must agree before anything is timed
+    if not (np.array_equal(tables.cpu().numpy(), tables1) and
+            np.array_equal(slots.cpu().numpy(), slots1) and
+            np.array_equal(qsl.cpu().numpy(), qsl1) and
+            np.array_equal(seq_lens.cpu().numpy(), nc + ql) and
+            state.cpu().tolist()[:3] == [head0 + per_call, 0, 0]):
+        raise RuntimeError("pa_plan_step and the host planner disagree")
+    # every call repeats the step (same counts, the next blocks of the queue)
+    left = len(step.free_queue) - head0 - per_call
+    n = int(max(1, min(args.steps, left // max(1, per_call) - args.warmup)))
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    dev_us = timed_loop([call], stream, n) * 1e3
+    if state[1].item() != 0:
+        raise RuntimeError("pa_plan_step refused a timed call")
+
+    pin = lambda a: torch.empty(a.shape, dtype=torch.from_numpy(a[:0]).dtype).pin_memory()
+    h_tab, h_slots, h_qsl, h_sl = pin(tables1), pin(slots1), pin(qsl1), pin(nc)
+    host_us = []
+    for _ in range(20):
+        pool = host_pool()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for s in range(S):
+            pool.allocate_slots(s, int(nc[s] + ql[s]))
+        tab = pool.block_table(range(S), mb)
+        sm = block_pool.slot_mapping(tab, nc, ql)
+        qs = block_pool.query_start_loc(ql)
+        h_tab.numpy()[...] = tab
+        h_slots.numpy()[...] = sm
+        h_qsl.numpy()[...] = qs
+        h_sl.numpy()[...] = nc + ql
+        tables.copy_(h_tab, non_blocking=True)
+        slots.copy_(h_slots, non_blocking=True)
+        qsl.copy_(h_qsl, non_blocking=True)
+        seq_lens.copy_(h_sl, non_blocking=True)
+        stream.synchronize()
+        host_us.append((time.perf_counter() - t0) * 1e6)
+    return {"workload": WORKLOAD, "num_seqs": S, "new_tokens": int(ql.sum()),
+            "blocks_taken_per_call": per_call,
+            "device_us_per_call": round(dev_us, 3), "calls": n,
+            "device_timing": "back-to-back pa_plan_step calls, CUDA events around the loop",
+            "host_us_per_step": round(statistics.median(host_us), 1),
+            "host_path": ("BlockPool.allocate_slots per sequence, block_table, slot_mapping, "
+                          "query_start_loc, four pinned copies to the device, stream sync "
+                          "(median of 20)"),
+            "equal_outputs": True}
+
+
 def bench_ours(args) -> None:
     import numpy as np
     import torch
@@ -453,6 +545,7 @@ def bench_ours(args) -> None:
     del dss, host_ins, ds0, step_graphs, attn_graphs, e2e_graphs
     torch.cuda.empty_cache()
     mixed = None if args.no_mixed else bench_mixed(args, dev, stream, world, clocks)
+    planner = None if args.no_planner or rank != 0 else bench_planner(args, dev, stream)
     clk = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -500,6 +593,7 @@ def bench_ours(args) -> None:
             "attention_graph_replay_ms": round(attn_graph_ms, 5),
             "gpu_launches": args.steps,
             "mixed_step": mixed,
+            "plan_step": planner,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clk}
@@ -518,6 +612,8 @@ def main(argv=None) -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mixed", action="store_true",
                     help="skip the mixed prefill+decode leg (Llama-3-8B shape)")
+    ap.add_argument("--no-planner", action="store_true",
+                    help="skip the on-GPU step planner measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

@@ -239,6 +239,65 @@ int pa_attention_varlen_static_scratch(
     int num_blocks, float scale, pa_dtype dtype, const int32_t* seq_lens_host,
     const int32_t* query_start_loc_host, struct CUstream_st* stream);
 
+/*
+ * pa_plan_step -- one scheduler step's block allocation and attention inputs,
+ * computed on the GPU (no host round trip between the steps of a decode loop).
+ *
+ * Page "LLM推論エンジンvLLMの内部構造を徹底解説", section "PagedAttentionの仕組み":
+ * a request of n tokens holds ceil(n / 16) blocks, and allocate_slots takes
+ * the blocks a request lacks from the front of free_block_queue into the
+ * request's block list, requests in order; the step's sequences form one
+ * super-sequence; a token at position p is stored in slot
+ * block_table[p / 16] * 16 + p % 16.  (Step 2 of allocate_slots, preempting
+ * requests when the pool runs dry, is scheduler policy: here a step that does
+ * not fit is refused, see the status bits.)
+ *
+ * Sequence s already owns the blocks of its first num_computed[s] tokens
+ * (entries 0 .. ceil(num_computed[s] / 16) - 1 of its row) and schedules
+ * query_lens[s] new tokens.  The call writes
+ *   seq_lens[s]        = num_computed[s] + query_lens[s]
+ *   query_start_loc    = 0, then the running sum of query_lens  ([num_seqs + 1])
+ *   block_tables[s][c] for c = ceil(num_computed[s] / 16) .. ceil(seq_lens[s] / 16) - 1:
+ *                        the next queue entries, sequences in order, from the
+ *                        queue head on (other entries are left as they are)
+ *   slot_mapping[query_start_loc[s] + j] = slot of position num_computed[s] + j
+ * and advances the queue head by the number of blocks taken.  These are the
+ * arguments pa_reshape_and_cache and pa_attention_varlen(_write_cache) take
+ * (with num_tokens = the sum of query_lens).
+ *
+ *   free_queue      int32 [queue_len]: block ids, front first
+ *   planner_state   int32 [4], 16-byte aligned, caller-owned: [0] queue head
+ *                   (index of the front entry, in and out), [1] status bits
+ *                   (sticky: set, never cleared, by the call), [2] used inside
+ *                   the call, must be 0 between calls, [3] unused.  Zero it
+ *                   once, then set [0] to where the queue's free part starts.
+ *   num_computed,
+ *   query_lens      int32 [num_seqs] (device; e.g. the previous step's
+ *                   seq_lens as num_computed)
+ *   block_tables    int32 [num_seqs][max_blocks_per_seq], updated in place
+ *   seq_lens        int32 [num_seqs] (written)
+ *   query_start_loc int32 [num_seqs + 1] (written)
+ *   slot_mapping    int64 [max_tokens] (the first sum(query_lens) written)
+ *
+ * Status bits, set on the device (read planner_state[1] after the stream
+ * has run; when any bit is set by a call, that call wrote nothing else and
+ * left the head as it was):
+ *   1  the queue holds fewer blocks than the step needs
+ *   2  a sequence would need more than max_blocks_per_seq blocks
+ *   4  sum(query_lens) > max_tokens
+ *   8  a negative count, or a sequence longer than INT32_MAX tokens
+ *  16  the queue head is outside [0, queue_len]
+ * Supported: block_size 16; num_seqs up to 16384 (more returns
+ * PA_ERR_UNSUPPORTED).  Entries of a row below num_computed's blocks are read
+ * for the slots but not checked against the pool (pa_reshape_and_cache skips
+ * slots outside it).
+ */
+int pa_plan_step(const int32_t* free_queue, int queue_len, int32_t* planner_state,
+                 const int32_t* num_computed, const int32_t* query_lens, int num_seqs,
+                 int32_t* block_tables, int max_blocks_per_seq, int block_size,
+                 int32_t* seq_lens, int32_t* query_start_loc, int64_t* slot_mapping,
+                 int max_tokens, struct CUstream_st* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -100,6 +100,32 @@ extern "C" int pa_reshape_and_cache(const void* k, const void* v, void* k_cache,
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+static bool aligned_to(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+extern "C" int pa_plan_step(const int32_t* free_queue, int queue_len, int32_t* planner_state,
+                            const int32_t* num_computed, const int32_t* query_lens,
+                            int num_seqs, int32_t* block_tables, int max_blocks_per_seq,
+                            int block_size, int32_t* seq_lens, int32_t* query_start_loc,
+                            int64_t* slot_mapping, int max_tokens, struct CUstream_st* stream) {
+  if (queue_len < 0 || num_seqs < 0 || max_blocks_per_seq < 0 || max_tokens < 0)
+    return PA_ERR_INVALID;
+  if (block_size != kBlockSize || num_seqs > kPlanMaxSeqs) return PA_ERR_UNSUPPORTED;
+  if (!planner_state || !query_start_loc) return PA_ERR_INVALID;
+  if (num_seqs > 0 && (!num_computed || !query_lens || !block_tables || !seq_lens))
+    return PA_ERR_INVALID;
+  if ((queue_len > 0 && !free_queue) || (max_tokens > 0 && !slot_mapping)) return PA_ERR_INVALID;
+  if (!aligned_to(planner_state, 16) || !aligned_to(query_start_loc, 4) ||
+      !aligned_to(num_computed, 4) || !aligned_to(query_lens, 4) ||
+      !aligned_to(block_tables, 4) || !aligned_to(seq_lens, 4) || !aligned_to(free_queue, 4) ||
+      !aligned_to(slot_mapping, 8))
+    return PA_ERR_INVALID;
+  cudaError_t e = launch_plan_step(free_queue, queue_len, planner_state, num_computed,
+                                   query_lens, num_seqs, block_tables, max_blocks_per_seq,
+                                   seq_lens, query_start_loc, slot_mapping, max_tokens,
+                                   (cudaStream_t)stream);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 extern "C" size_t pa_attention_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                               int head_dim, int max_seq_len) {
   if (num_seqs < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_seq_len < 0) return 0;

@@ -127,4 +127,22 @@ cudaError_t launch_prefill_tcgen05(const AttnParams& p, int head_dim, int max_qu
                                    int num_items, const int32_t* seq_lens_host,
                                    const int32_t* query_start_loc_host, cudaStream_t stream);
 
+// On-GPU step planner (allocate_slots, seq_lens, query_start_loc, slot
+// mapping).  planner state: int32[4] in device memory.
+constexpr int kPlanStateHead = 0;      // index of the queue's front entry
+constexpr int kPlanStateStatus = 1;    // error bits below (sticky)
+constexpr int kPlanStateArrivals = 2;  // CTAs done with the current launch (0 between calls)
+constexpr int kPlanMaxSeqs = 16384;    // sequences one call plans (their sums sit in shared memory)
+constexpr int kPlanPoolEmpty = 1;      // the queue holds fewer blocks than the step needs
+constexpr int kPlanRowFull = 2;        // a sequence would outgrow its block-table row
+constexpr int kPlanSlotsFull = 4;      // more scheduled tokens than slot_mapping holds
+constexpr int kPlanBadLength = 8;      // a negative count, or a length past int32
+constexpr int kPlanBadHead = 16;       // the queue head lies outside the queue
+size_t plan_step_smem(int num_seqs);
+cudaError_t launch_plan_step(const int32_t* free_queue, int queue_len, int32_t* state,
+                             const int32_t* num_computed, const int32_t* query_lens,
+                             int num_seqs, int32_t* block_tables, int max_blocks_per_seq,
+                             int32_t* seq_lens, int32_t* query_start_loc,
+                             int64_t* slot_mapping, int max_tokens, cudaStream_t stream);
+
 }  // namespace pa

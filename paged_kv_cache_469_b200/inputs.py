@@ -236,3 +236,19 @@ def random_step(seed: int, *, dtype: str = "bf16", num_q_heads: int = 8, num_kv_
                      num_kv_heads=num_kv_heads, head_dim=head_dim, num_blocks=num_blocks,
                      seq_lens=lens, query_lens=qls, seed=seed, rng=rng,
                      shared_prefix_tokens=shared_prefix_tokens)
+
+
+def planner_draws(seed: int, *, num_seqs: int, num_blocks: int, max_ctx: int = 4096,
+                  max_chunk: int = 512, prefill_frac: float = 0.1, idle_frac: float = 0.05):
+    """Draws for one scheduler step of the block planner: a shuffled
+    free_block_queue, the tokens each sequence already holds blocks for, and
+    the tokens it schedules now (mostly one-token decodes, some prefill chunks
+    of 2..max_chunk tokens, a few sequences with nothing scheduled)."""
+    rng = np.random.default_rng([seed, 7])
+    free_queue = rng.permutation(num_blocks).astype(np.int32)
+    num_computed = rng.integers(0, max_ctx, size=num_seqs, endpoint=True).astype(np.int32)
+    kind = rng.random(num_seqs)
+    chunk = rng.integers(2, max(2, max_chunk), size=num_seqs, endpoint=True)
+    query_lens = np.where(kind < idle_frac, 0,
+                          np.where(kind < idle_frac + prefill_frac, chunk, 1)).astype(np.int32)
+    return free_queue, num_computed, query_lens

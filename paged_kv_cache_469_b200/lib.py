@@ -21,7 +21,8 @@ PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
 # every symbol include/pa.h declares
 EXPORTS = ("pa_status_string", "pa_reshape_and_cache", "pa_attention_workspace_size",
            "pa_workspace_init", "pa_workspace_status", "pa_attention_varlen",
-           "pa_attention_varlen_write_cache", "pa_attention_varlen_static_scratch")
+           "pa_attention_varlen_write_cache", "pa_attention_varlen_static_scratch",
+           "pa_plan_step")
 
 _lib = None
 
@@ -60,6 +61,9 @@ def library() -> ctypes.CDLL:
         lib.pa_attention_varlen_write_cache.argtypes = [
             c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_int, c_p, c_p, c_int, c_int, c_int, c_int,
             c_int, c_int, c_int, c_int, c_int, c_f, c_int, c_p, c_sz, c_p, c_p, c_p]
+        lib.pa_plan_step.restype = c_int
+        lib.pa_plan_step.argtypes = [c_p, c_int, c_p, c_p, c_p, c_int, c_p, c_int, c_int, c_p,
+                                     c_p, c_p, c_int, c_p]
         _lib = lib
     return _lib
 
@@ -196,3 +200,43 @@ def attention_varlen_write_cache(out: torch.Tensor, q: torch.Tensor, k_new: torc
     if rc != PA_OK:
         raise PAError(rc, "pa_attention_varlen_write_cache")
     return out
+
+
+# bits of planner_state[1] (see pa_plan_step in pa.h)
+PLAN_POOL_EMPTY, PLAN_ROW_FULL, PLAN_SLOTS_FULL, PLAN_BAD_LENGTH, PLAN_BAD_HEAD = 1, 2, 4, 8, 16
+
+
+def new_planner_state(queue_head: int = 0, device="cuda") -> torch.Tensor:
+    """int32[4] planner state: queue head, status bits, two words the call uses."""
+    st = torch.zeros(4, dtype=torch.int32, device=device)
+    st[0] = queue_head
+    return st
+
+
+def plan_step(free_queue: torch.Tensor, planner_state: torch.Tensor,
+              num_computed: torch.Tensor, query_lens: torch.Tensor, block_tables: torch.Tensor,
+              seq_lens: torch.Tensor, query_start_loc: torch.Tensor,
+              slot_mapping: torch.Tensor, block_size: int = 16, stream=None) -> None:
+    """Block allocation, seq_lens, query_start_loc and slot mapping of one step on
+    the GPU (see pa_plan_step in pa.h); errors land in planner_state[1]."""
+    for name, t in (("free_queue", free_queue), ("planner_state", planner_state),
+                    ("num_computed", num_computed), ("query_lens", query_lens),
+                    ("block_tables", block_tables), ("seq_lens", seq_lens),
+                    ("query_start_loc", query_start_loc)):
+        if t.dtype != torch.int32:
+            raise TypeError(f"{name} must be int32")
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    num_seqs = query_lens.shape[0]
+    if num_computed.shape[0] != num_seqs or seq_lens.shape[0] != num_seqs or \
+            query_start_loc.shape[0] != num_seqs + 1 or block_tables.shape[0] != num_seqs or \
+            planner_state.numel() != 4:
+        raise ValueError("plan_step: inconsistent sizes")
+    rc = library().pa_plan_step(
+        _dev(free_queue, "free_queue"), free_queue.numel(), _dev(planner_state, "planner_state"),
+        _dev(num_computed, "num_computed"), _dev(query_lens, "query_lens"), num_seqs,
+        _dev(block_tables, "block_tables"), block_tables.shape[1], block_size,
+        _dev(seq_lens, "seq_lens"), _dev(query_start_loc, "query_start_loc"),
+        _dev(slot_mapping, "slot_mapping"), slot_mapping.numel(), _stream(stream))
+    if rc != PA_OK:
+        raise PAError(rc, "pa_plan_step")

@@ -125,6 +125,32 @@ def test_reshape_argument_checks(L):
     assert f(0, 0, 0, 0, 0, 0, 2, 64, 16, 8, 1, None) == palib.PA_OK
 
 
+def _plan(L, **kw):
+    args = dict(fq=16, qlen=64, state=16, nc=16, ql=16, S=2, bt=16, mb=8, bs=16, sl=16,
+                qsl=16, slots=16, cap=8, stream=None)
+    args.update(kw)
+    return L.pa_plan_step(*args.values())
+
+
+def test_plan_step_argument_checks(L):
+    """pa_plan_step rejects bad sizes, pointers and alignments on the host."""
+    assert _plan(L, bs=32) == palib.PA_ERR_UNSUPPORTED
+    assert _plan(L, S=16385) == palib.PA_ERR_UNSUPPORTED  # more sequences than one call plans
+    assert _plan(L, S=-1) == palib.PA_ERR_INVALID
+    assert _plan(L, qlen=-1) == palib.PA_ERR_INVALID
+    assert _plan(L, mb=-1) == palib.PA_ERR_INVALID
+    assert _plan(L, cap=-1) == palib.PA_ERR_INVALID
+    assert _plan(L, state=0) == palib.PA_ERR_INVALID
+    assert _plan(L, state=8) == palib.PA_ERR_INVALID     # state not 16-byte aligned
+    assert _plan(L, qsl=0) == palib.PA_ERR_INVALID
+    assert _plan(L, nc=0) == palib.PA_ERR_INVALID
+    assert _plan(L, bt=0) == palib.PA_ERR_INVALID
+    assert _plan(L, fq=0) == palib.PA_ERR_INVALID        # a queue of 64 entries at NULL
+    assert _plan(L, slots=0) == palib.PA_ERR_INVALID     # room for 8 slots at NULL
+    assert _plan(L, slots=20) == palib.PA_ERR_INVALID    # int64 slots misaligned
+    assert _plan(L, ql=18) == palib.PA_ERR_INVALID       # int32 array misaligned
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(palib, "_lib", None)
     monkeypatch.setattr(palib, "LIB_PATH", str(tmp_path / "nope.so"))
