@@ -111,14 +111,15 @@ cudaError_t launch_reshape_and_cache(const void* k, const void* v, void* k_cache
 cudaError_t launch_attention_simple(const AttnParams& p, int head_dim, bool is_bf16,
                                     int min_rows_per_kv_head, cudaStream_t stream);
 
-// Split-K decode kernel (bf16): sequences with q_len * group <= 16.
+// Split-K decode kernel (bf16): sequences with q_len * group <= kDecodeMaxRows (64),
+// in 16-row groups.
 // Decode CTAs the GPU holds at once for this head_dim and query-row count
 // (SMs x resident CTAs per SM); looked up once per device and shape.
 int decode_wave_ctas(int head_dim, int rows);
 cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
                                  cudaStream_t stream);
 
-// Tensor-core prefill kernel (bf16): sequences with q_len * group > 16.
+// Tensor-core prefill kernel (bf16): sequences with q_len * group > kDecodeMaxRows.
 // num_items >= 0: the work list in ws_items was written by the host (exact
 // count); num_items < 0: build it on the device first.
 constexpr int kPrefillQTile = 128;  // query rows per Q tile (MMA M); a work item holds two
