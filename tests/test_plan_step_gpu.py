@@ -20,6 +20,7 @@ import torch
 import oracle
 from paged_kv_cache_469_b200 import lib
 from paged_kv_cache_469_b200.inputs import planner_draws
+from tests.oracle_side import oracle_plan_step
 
 pytestmark = pytest.mark.gpu
 
@@ -28,20 +29,7 @@ PAD = -7  # entries no call should touch
 
 def expected_step(free_queue, head, tables, num_computed, query_lens):
     """(tables, seq_lens, query_start_loc, slots, new head) one call must give."""
-    need = np.array([oracle.blocks_needed(int(c) + int(q)) - oracle.blocks_needed(int(c))
-                     for c, q in zip(num_computed, query_lens)], dtype=np.int64)
-    new_rows, taken = oracle.allocate_block_tables(
-        free_queue[head:], (need * 16).astype(np.int32),
-        max_blocks_per_seq=max(1, int(need.max(initial=0))), pad_value=PAD)
-    out = tables.copy()
-    for s in range(len(need)):
-        first = oracle.blocks_needed(int(num_computed[s]))
-        assert first + need[s] <= out.shape[1], "the case outgrows its table"
-        out[s, first:first + need[s]] = new_rows[s, :need[s]]
-    seq_lens = (num_computed.astype(np.int64) + query_lens).astype(np.int32)
-    qsl = oracle.query_start_loc(query_lens)
-    slots = oracle.slot_mapping(out, num_computed, query_lens)
-    return out, seq_lens, qsl, slots, head + taken
+    return oracle_plan_step(free_queue, head, tables, num_computed, query_lens, pad_value=PAD)
 
 
 class Planner:
