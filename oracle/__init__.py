@@ -59,6 +59,9 @@ def _load():
         lib.oracle_query_start_loc.argtypes = [c_p, c_int, c_p]
         lib.oracle_slot_mapping.restype = c_int
         lib.oracle_slot_mapping.argtypes = [c_p, c_int, c_int, c_p, c_p, c_int, c_p]
+        lib.oracle_plan_step.restype = c_int
+        lib.oracle_plan_step.argtypes = [c_p, c_i64, c_p, c_p, c_p, c_int, c_p, c_int, c_int,
+                                         c_p, c_p, c_p, c_i64]
         lib.oracle_reshape_and_cache.restype = None
         lib.oracle_reshape_and_cache.argtypes = [c_p, c_p, c_p, c_p, c_p, c_i64, c_int, c_int,
                                                  c_int, c_int]
@@ -131,6 +134,31 @@ def slot_mapping(block_tables: np.ndarray, first_pos: np.ndarray, count: np.ndar
     if rc != 0:
         raise ValueError("oracle slot mapping: position beyond the block table")
     return out
+
+
+def plan_step(free_queue: np.ndarray, head: int, block_tables: np.ndarray,
+              num_computed: np.ndarray, query_lens: np.ndarray, *, block_size: int = 16,
+              max_tokens: int | None = None):
+    """One scheduler step of block planning (allocate_slots for a running batch)
+    -> (block_tables, seq_lens, query_start_loc, slots, new head); the input
+    table is not modified.  Raises ValueError when the step does not fit."""
+    fq = np.ascontiguousarray(free_queue, dtype=np.int32)
+    nc = np.ascontiguousarray(num_computed, dtype=np.int32)
+    ql = np.ascontiguousarray(query_lens, dtype=np.int32)
+    tables = np.array(block_tables, dtype=np.int32, copy=True, order="C")
+    s = len(ql)
+    seq_lens = np.empty(s, dtype=np.int32)
+    qsl = np.empty(s + 1, dtype=np.int32)
+    total = int(np.maximum(ql, 0).sum())
+    cap = total if max_tokens is None else int(max_tokens)
+    slots = np.empty(max(total, 1), dtype=np.int64)
+    h = ctypes.c_int64(int(head))
+    rc = _load().oracle_plan_step(_ptr(fq), len(fq), ctypes.addressof(h), _ptr(nc), _ptr(ql), s,
+                                  _ptr(tables), tables.shape[1], block_size, _ptr(seq_lens),
+                                  _ptr(qsl), _ptr(slots), cap)
+    if rc != 0:
+        raise ValueError("oracle plan_step: the step does not fit (pool, row, slots or counts)")
+    return tables, seq_lens, qsl, slots[:total], int(h.value)
 
 
 def reshape_and_cache(k: np.ndarray, v: np.ndarray, k_cache: np.ndarray,

@@ -36,8 +36,9 @@
  * contiguous K/V (a library routine), permutation invariance of physical block
  * ids, closed-form special cases (one key, constant V, zero query), GQA equal to
  * MHA with repeated KV heads, chunked prefill equal to one-shot prefill, a
- * shared prefix equal to private copies, and an exhaustive check of the bf16
- * rounding against exact rational arithmetic.
+ * shared prefix equal to private copies, an exhaustive check of the bf16
+ * rounding against exact rational arithmetic, and the step planner against
+ * allocate_slots walked by hand over chained steps.
  */
 #include <math.h>
 #include <stdint.h>
@@ -146,6 +147,56 @@ int oracle_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq,
       slots[out++] = phys * block_size + offset;
     }
   }
+  return 0;
+}
+
+/* One scheduler step of block planning for a running batch.  Sequence s
+ * holds the blocks of its first num_computed[s] tokens (the first
+ * blocks_needed(num_computed[s]) entries of its row) and schedules
+ * query_lens[s] new tokens.  allocate_slots, sequences in order: each takes
+ * the blocks it still lacks for num_computed[s] + query_lens[s] tokens from
+ * the front of the queue (which starts at *head) and appends them to its row.
+ * Then seq_lens[s] = num_computed[s] + query_lens[s], the super-sequence
+ * offsets of query_lens, and the slot of every new position num_computed[s] ..
+ * seq_lens[s] - 1, in order.
+ *
+ * The whole step is checked before anything is written: a negative count, a
+ * head outside the queue, a row that would grow past max_blocks_per_seq, a
+ * queue that runs dry or more new tokens than max_tokens returns -1 and
+ * writes nothing.  On success *head has moved past the blocks taken. */
+int oracle_plan_step(const int32_t* free_queue, int64_t queue_len, int64_t* head,
+                     const int32_t* num_computed, const int32_t* query_lens, int num_seqs,
+                     int32_t* block_tables, int max_blocks_per_seq, int block_size,
+                     int32_t* seq_lens, int32_t* query_start_loc, int64_t* slots,
+                     int64_t max_tokens) {
+  int64_t wanted = 0, tokens = 0;
+  if (*head < 0 || *head > queue_len) return -1;
+  for (int s = 0; s < num_seqs; ++s) {
+    if (num_computed[s] < 0 || query_lens[s] < 0) return -1;
+    int64_t len = (int64_t)num_computed[s] + query_lens[s];
+    if (len > INT32_MAX) return -1;
+    int64_t have = oracle_blocks_needed(num_computed[s], block_size);
+    int64_t need = oracle_blocks_needed(len, block_size);
+    if (need > max_blocks_per_seq) return -1;
+    wanted += need - have;
+    tokens += query_lens[s];
+  }
+  if (wanted > queue_len - *head || tokens > max_tokens) return -1;
+
+  int64_t next = *head;
+  for (int s = 0; s < num_seqs; ++s) {
+    int32_t* row = block_tables + (int64_t)s * max_blocks_per_seq;
+    int64_t len = (int64_t)num_computed[s] + query_lens[s];
+    int64_t have = oracle_blocks_needed(num_computed[s], block_size);
+    int64_t need = oracle_blocks_needed(len, block_size);
+    for (int64_t c = have; c < need; ++c) row[c] = free_queue[next++];
+    seq_lens[s] = (int32_t)len;
+  }
+  oracle_query_start_loc(query_lens, num_seqs, query_start_loc);
+  if (oracle_slot_mapping(block_tables, max_blocks_per_seq, num_seqs, num_computed, query_lens,
+                          block_size, slots) != 0)
+    return -1; /* unreachable after the row check */
+  *head = next;
   return 0;
 }
 

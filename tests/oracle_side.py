@@ -29,30 +29,6 @@ def oracle_state(step: StepInputs, max_blocks_per_seq: int | None = None, pad_va
                 slot_mapping=new_slots, ctx_slot_mapping=ctx_slots, k_cache=kc, v_cache=vc)
 
 
-def oracle_plan_step(free_queue, head: int, tables, num_computed, query_lens,
-                     pad_value: int = 0):
-    """One scheduler step of block planning, from the oracle's own steps:
-    every sequence takes, in order, from the queue front at `head`, the blocks
-    its new tokens add (allocate_slots of blocks_needed(new length) minus
-    blocks_needed(old length)), appended after the blocks it holds; then the
-    step's query_start_loc and the slots of the new positions.
-    Returns (tables, seq_lens, query_start_loc, slots, new head)."""
-    need = np.array([oracle.blocks_needed(int(c) + int(q)) - oracle.blocks_needed(int(c))
-                     for c, q in zip(num_computed, query_lens)], dtype=np.int64)
-    new_rows, taken = oracle.allocate_block_tables(
-        np.asarray(free_queue)[head:], (need * 16).astype(np.int32),
-        max_blocks_per_seq=max(1, int(need.max(initial=0))), pad_value=pad_value)
-    out = np.array(tables, dtype=np.int32, copy=True)
-    for s in range(len(need)):
-        first = oracle.blocks_needed(int(num_computed[s]))
-        assert first + need[s] <= out.shape[1], "the case outgrows its table"
-        out[s, first:first + need[s]] = new_rows[s, :need[s]]
-    seq_lens = (np.asarray(num_computed, dtype=np.int64) + query_lens).astype(np.int32)
-    qsl = oracle.query_start_loc(query_lens)
-    slots = oracle.slot_mapping(out, num_computed, query_lens)
-    return out, seq_lens, qsl, slots, head + taken
-
-
 def oracle_outputs(step: StepInputs, state=None, num_threads: int = 1) -> np.ndarray:
     st = state or oracle_state(step)
     return oracle.paged_attention(step.q, st["k_cache"], st["v_cache"], st["block_tables"],

@@ -43,6 +43,17 @@ MUTANTS = [
      "int64_t b = t / block_size;\n    int o = (int)(t % block_size);\n    double dot"),
     ("bf16_ties_away", "if (frac > 0.5 || (frac == 0.5 && fmod(ip, 2.0) != 0.0)) ip += 1.0;",
      "if (frac >= 0.5) ip += 1.0;"),
+    ("plan_overwrites_held_blocks",
+     "for (int64_t c = have; c < need; ++c) row[c] = free_queue[next++];",
+     "for (int64_t c = 0; c < need - have; ++c) row[c] = free_queue[next++];"),
+    ("plan_slots_from_new_length",
+     "if (oracle_slot_mapping(block_tables, max_blocks_per_seq, num_seqs, num_computed, "
+     "query_lens,",
+     "if (oracle_slot_mapping(block_tables, max_blocks_per_seq, num_seqs, seq_lens, "
+     "query_lens,"),
+    ("plan_head_not_advanced", "  *head = next;\n  return 0;", "  return 0;"),
+    ("plan_pool_check_off_by_one", "if (wanted > queue_len - *head || tokens > max_tokens)",
+     "if (wanted >= queue_len - *head || tokens > max_tokens)"),
 ]
 
 

@@ -20,7 +20,7 @@ import pytest
 import torch
 
 import oracle
-from paged_kv_cache_469_b200.inputs import make_step, random_step, workload
+from paged_kv_cache_469_b200.inputs import make_step, planner_draws, random_step, workload
 from tests.oracle_side import as_f64, contiguous_kv, oracle_outputs, oracle_state
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -314,13 +314,138 @@ def check_workload_block_counts():
     assert list(state["block_tables"][0, :2]) == list(st.free_queue[:2])
 
 
+# ---------------------------------------------------------------- step planning
+#
+# oracle.plan_step against allocate_slots walked by hand: a Python list for the
+# queue, one block per started group of 16 tokens counted token by token, the
+# slot of position p read from the row at p // 16, offset p % 16 -- no block
+# arithmetic shared with the oracle.
+
+PLAN_PAD = -3
+
+
+def _hand_walk(free_queue, steps):
+    """Per step: (rows, seq_lens, query_start_loc, slots, head)."""
+    queue = [int(b) for b in free_queue]
+    taken = 0
+    rows: dict = {}
+    for num_computed, query_lens in steps:
+        seq_lens, qsl, slots = [], [0], []
+        for s in range(len(query_lens)):
+            row = rows.setdefault(s, [])
+            length = int(num_computed[s]) + int(query_lens[s])
+            started = sum(1 for t in range(length) if t % 16 == 0)
+            while len(row) < started:
+                row.append(queue[taken])
+                taken += 1
+            seq_lens.append(length)
+            qsl.append(qsl[-1] + int(query_lens[s]))
+            for j in range(int(query_lens[s])):
+                p = int(num_computed[s]) + j
+                slots.append(row[p // 16] * 16 + p % 16)
+        yield ({s: list(r) for s, r in rows.items()}, np.array(seq_lens), np.array(qsl),
+               np.array(slots, dtype=np.int64), taken)
+
+
+def _rows_match(tables, rows):
+    for s, r in rows.items():
+        assert tables[s, :len(r)].tolist() == r, f"row {s}"
+        assert (tables[s, len(r):] == PLAN_PAD).all(), f"row {s} written past its blocks"
+
+
+def check_plan_step_fresh_is_whole_allocation():
+    for S in (1, 6, 57):
+        fq, _, ql = planner_draws(100 + S, num_seqs=S, num_blocks=5000, max_ctx=0,
+                                  max_chunk=300, prefill_frac=0.6)
+        nc = np.zeros(S, np.int32)
+        tables, sl, qsl, slots, head = oracle.plan_step(
+            fq, 0, np.full((S, 32), PLAN_PAD, np.int32), nc, ql)
+        whole, taken = oracle.allocate_block_tables(fq, ql, max_blocks_per_seq=32,
+                                                    pad_value=PLAN_PAD)
+        np.testing.assert_array_equal(tables, whole)
+        assert head == taken
+        (rows, w_sl, w_qsl, w_slots, w_head), = _hand_walk(fq, [(nc, ql)])
+        _rows_match(tables, rows)
+        np.testing.assert_array_equal(slots, w_slots)
+        np.testing.assert_array_equal(qsl, w_qsl)
+        np.testing.assert_array_equal(sl, w_sl)
+
+
+def check_plan_step_chained_steps():
+    """A context allocation, then five steps of decodes, chunks and idle
+    sequences, each starting where the previous one left the queue."""
+    for seed in (1, 2, 3):
+        S = 23
+        fq, nc0, ql = planner_draws(seed, num_seqs=S, num_blocks=4000, max_ctx=300,
+                                    max_chunk=70, prefill_frac=0.3, idle_frac=0.2)
+        rng = np.random.default_rng(seed)
+        steps = [(np.zeros(S, np.int32), nc0)]
+        nc = nc0
+        for _ in range(5):
+            steps.append((nc, ql))
+            nc = (nc + ql).astype(np.int32)
+            ql = np.where(rng.random(S) < 0.3, rng.integers(0, 50, S), 1).astype(np.int32)
+        tables = np.full((S, 64), PLAN_PAD, np.int32)
+        head = 0
+        for (num_computed, query_lens), walk in zip(steps, _hand_walk(fq, steps)):
+            tables, sl, qsl, slots, head = oracle.plan_step(fq, head, tables, num_computed,
+                                                            query_lens)
+            rows, w_sl, w_qsl, w_slots, w_head = walk
+            _rows_match(tables, rows)
+            np.testing.assert_array_equal(sl, w_sl)
+            np.testing.assert_array_equal(qsl, w_qsl)
+            np.testing.assert_array_equal(slots, w_slots)
+            assert head == w_head
+
+
+def check_plan_step_invariants():
+    """One step's slots are distinct, each lies in a block of its own
+    sequence's row, and the blocks appended are the queue entries taken."""
+    S = 40
+    fq, nc, ql = planner_draws(9, num_seqs=S, num_blocks=6000, max_ctx=500, max_chunk=100,
+                               prefill_frac=0.4)
+    tables0, head0 = oracle.allocate_block_tables(fq, nc, max_blocks_per_seq=64,
+                                                  pad_value=PLAN_PAD)
+    tables, _, qsl, slots, head = oracle.plan_step(fq, head0, tables0, nc, ql)
+    assert len(set(slots.tolist())) == len(slots)
+    for s in range(S):
+        own = set(tables[s][tables[s] != PLAN_PAD].tolist())
+        assert {int(x) // 16 for x in slots[qsl[s]:qsl[s + 1]]} <= own
+    appended = sorted(set(tables[tables != PLAN_PAD].tolist()) -
+                      set(tables0[tables0 != PLAN_PAD].tolist()))
+    assert appended == sorted(fq[head0:head].tolist())
+
+
+def check_plan_step_refusals():
+    """A step that does not fit is refused as a whole; the limits themselves fit."""
+    fq = np.arange(10, dtype=np.int32)
+    t = np.full((2, 4), PLAN_PAD, np.int32)
+    nc = np.array([16, 0], np.int32)
+    ok = oracle.plan_step(fq, 1, t, nc, np.array([48, 64], np.int32))  # rows exactly full
+    assert ok[4] == 1 + 3 + 4
+    for head, ql, cap in ((3, [48, 64], None),   # 7 blocks wanted, 7 left: fits ...
+                          (4, [48, 64], None),   # ... 6 left: pool runs dry
+                          (0, [49, 0], None),    # row 0 would need a 5th block
+                          (0, [1, -1], None),    # negative count
+                          (11, [1, 1], None),    # head past the queue
+                          (0, [3, 4], 6)):       # 7 tokens, room for 6
+        try:
+            oracle.plan_step(fq, head, t, nc, np.array(ql, np.int32), max_tokens=cap)
+            refused = False
+        except ValueError:
+            refused = True
+        assert refused == (head != 3), (head, ql, cap)
+
+
 CHECKS = [check_worked_example, check_blocks_needed_brute_force,
           check_allocation_pops_queue_front, check_shared_prefix_allocation,
           check_slot_mapping_brute_force, check_query_start_loc, check_reshape_and_cache,
           check_dense_agreement, check_block_permutation_invariance,
           check_sequence_reorder_invariance, check_special_cases, check_gqa_equals_repeated_mha,
           check_chunked_prefill_equals_one_shot, check_shared_prefix_equals_private_copies,
-          check_bf16_rounding_exhaustive, check_workload_block_counts]
+          check_bf16_rounding_exhaustive, check_workload_block_counts,
+          check_plan_step_fresh_is_whole_allocation, check_plan_step_chained_steps,
+          check_plan_step_invariants, check_plan_step_refusals]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])

@@ -1,15 +1,11 @@
 """The on-GPU step planner (pa_plan_step, through the C ABI) against the
 oracle's allocation, prefix sums and slot mapping, bit-exact.
 
-One planner call must equal, entry for entry:
-  - the new blocks of each sequence: the oracle's allocate_slots over the
-    queue from the current head, each sequence asking for the blocks its new
-    tokens add (blocks_needed(new length) - blocks_needed(old length));
-  - query_start_loc: the oracle's prefix sum of query_lens;
-  - slot_mapping: the oracle's slot mapping of positions num_computed ..
-    num_computed + query_lens - 1 through the updated table;
-  - the new queue head: the old one plus the blocks taken.
-A call that cannot fit sets its status bit and writes nothing else.
+One planner call must equal the oracle's plan_step entry for entry: the
+blocks each sequence appends (allocate_slots from the queue front at the
+current head, sequences in order), seq_lens, query_start_loc, the slots of the
+new positions, and the new queue head.  A call that cannot fit sets its status
+bit and writes nothing else.
 """
 from __future__ import annotations
 
@@ -20,7 +16,6 @@ import torch
 import oracle
 from paged_kv_cache_469_b200 import lib
 from paged_kv_cache_469_b200.inputs import planner_draws
-from tests.oracle_side import oracle_plan_step
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +24,7 @@ PAD = -7  # entries no call should touch
 
 def expected_step(free_queue, head, tables, num_computed, query_lens):
     """(tables, seq_lens, query_start_loc, slots, new head) one call must give."""
-    return oracle_plan_step(free_queue, head, tables, num_computed, query_lens, pad_value=PAD)
+    return oracle.plan_step(free_queue, head, tables, num_computed, query_lens)
 
 
 class Planner:
