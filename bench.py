@@ -385,8 +385,11 @@ def bench_planner(args, dev, stream) -> dict:
     qsl1 = block_pool.query_start_loc(ql)
     per_call = len(step.free_queue) - len(pool.free_block_queue) - head0
 
-    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-    fq, tables, nc_t, ql_t = t(step.free_queue), t(tables0), t(nc), t(ql)
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    fq, tables, nc_t, ql_t = (to_dev(step.free_queue), to_dev(tables0), to_dev(nc),
+                              to_dev(ql))
     state = lib.new_planner_state(head0, device=dev)
     seq_lens = torch.empty(S, dtype=torch.int32, device=dev)
     qsl = torch.empty(S + 1, dtype=torch.int32, device=dev)
@@ -414,8 +417,11 @@ def bench_planner(args, dev, stream) -> dict:
     if state[1].item() != 0:
         raise RuntimeError("pa_plan_step refused a timed call")
 
-    pin = lambda a: torch.empty(a.shape, dtype=torch.from_numpy(a[:0]).dtype).pin_memory()
-    h_tab, h_slots, h_qsl, h_sl = pin(tables1), pin(slots1), pin(qsl1), pin(nc)
+    def pinned_like(a):
+        return torch.from_numpy(np.empty_like(a)).pin_memory()
+
+    h_tab, h_slots, h_qsl, h_sl = (pinned_like(tables1), pinned_like(slots1), pinned_like(qsl1),
+                                   pinned_like(nc))
     host_us = []
     for _ in range(20):
         pool = host_pool()
