@@ -162,7 +162,9 @@ int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_s
  * Supported: head_dim in {64, 128}; block_size 16; num_q_heads a multiple of
  * num_kv_heads with at most 16 q-heads per kv-head; dtype f32 or bf16;
  * max_seq_len up to at least 1.5M tokens (a longer bound than the split-K
- * merge can hold returns PA_ERR_UNSUPPORTED).
+ * merge can hold returns PA_ERR_UNSUPPORTED); at most 65535 sequences in a
+ * bf16 call that may hold decode-class sequences (without the host copies,
+ * every bf16 call may), else PA_ERR_UNSUPPORTED.
  */
 int pa_attention_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
                         const int32_t* block_tables, int max_blocks_per_seq,

@@ -224,6 +224,9 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
   const WorkspaceLayout w =
       workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len);
   if (w.max_parts > kDecodeMaxParts) return PA_ERR_UNSUPPORTED;
+  // the decode grid holds one sequence per z index
+  if (any_decode && dtype == PA_DTYPE_BF16 && num_seqs > kDecodeMaxSeqs)
+    return PA_ERR_UNSUPPORTED;
   AttnParams p{};
   p.out = out;
   p.q = q;

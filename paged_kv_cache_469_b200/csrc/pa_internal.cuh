@@ -41,6 +41,8 @@ constexpr int kDecodeMaxRows = kDecodeRows * kDecodeRowGroups;
 // memory holds each partition's per-row max and sum): 1536 partitions of at
 // least 1024 keys, i.e. sequences of at least 1.5M tokens
 constexpr int kDecodeMaxParts = 1536;
+// sequences one decode launch covers (grid z)
+constexpr int kDecodeMaxSeqs = 65535;
 #ifndef PA_DECODE_WARPS
 #define PA_DECODE_WARPS 4
 #endif

@@ -73,6 +73,9 @@ def test_attention_argument_checks(L):
     assert _varlen(L, out=0) == palib.PA_ERR_INVALID
     assert _varlen(L, S=-1) == palib.PA_ERR_INVALID
     assert _varlen(L, T=0) == palib.PA_OK  # nothing to do, nothing launched
+    # more sequences than the decode grid holds (without host copies any
+    # sequence may be decode-class)
+    assert _varlen(L, S=65536, T=65536) == palib.PA_ERR_UNSUPPORTED
     # a bound past what the split-K merge can hold (1537 partitions of 2048 keys)
     assert _varlen(L, ms=1536 * 2048 + 1, mb=(1536 * 2048 + 1 + 15) // 16) == \
         palib.PA_ERR_UNSUPPORTED
