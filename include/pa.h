@@ -141,7 +141,10 @@ int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_s
  *                  seq_lens[s] are never used, whatever they hold.
  *   seq_lens       int32 [num_seqs]
  *   query_start_loc int32 [num_seqs + 1], query_start_loc[0] = 0,
- *                  nondecreasing, query_start_loc[num_seqs] = num_tokens
+ *                  nondecreasing, query_start_loc[num_seqs] = num_tokens.
+ *                  The kernels trust these device arrays as given (a
+ *                  malformed query_start_loc would index q and out out of
+ *                  range); the host copies below, when given, are checked
  *   max_query_len, max_seq_len  host-side upper bounds over the step (they
  *                  size the launch grids; a sequence beyond them is caller
  *                  error and may be left unwritten)
