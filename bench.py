@@ -38,6 +38,7 @@ WORKLOAD = "decode_tinyllama"
 MIXED_WORKLOAD = "mixed_llama3_8b"
 L2_BYTES = 126 * 1000 * 1000  # B200 L2, for sizing the rotation of workload copies
 MAX_COPIES = 8
+REFERENCE_BUDGET_S = 120.0  # host seconds the --impl reference steps may take in all
 # dram__bytes_read.sum + dram__bytes_write.sum of one decode_splitk_kernel<64,false,4,4,false>
 # launch on this workload, from an ncu --set full capture of that launch; set
 # to None whenever that kernel changes, until it is captured again
@@ -234,7 +235,10 @@ def bench_reference(args) -> None:
     from paged_kv_cache_469_b200.inputs import workload
     step = workload(WORKLOAD)
     threads = os.cpu_count() or 1
-    gbs, n, dt, run, _ = oracle_sample(step, target_s=1.0, threads=threads)
+    # each step a bounded sample: about 1 s, less when there are many steps, so
+    # that the whole run stays near two minutes of host time
+    per_step = min(1.0, REFERENCE_BUDGET_S / (args.steps + args.warmup))
+    gbs, n, dt, run, _ = oracle_sample(step, target_s=per_step, threads=threads)
     import numpy as np
     for _ in range(args.warmup):
         run(n)
