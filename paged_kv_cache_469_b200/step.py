@@ -4,10 +4,12 @@
 the host (block allocation, slot mapping, super-sequence offsets), puts the
 cache and the step's tensors in device memory, writes the earlier tokens' K/V
 into the cache with ``pa_reshape_and_cache``, and then runs the step itself:
-``pa_reshape_and_cache`` for the new tokens followed by
-``pa_attention_varlen``.  ``capture`` records those launches in a CUDA graph,
-the way a serving loop replays a steady decode step without paying the host
-cost of each call again.
+``run`` makes two calls (``pa_reshape_and_cache`` for the new tokens, then
+``pa_attention_varlen``), ``run_fused`` makes one
+(``pa_attention_varlen_write_cache``).  The step's inputs sit in one device
+buffer, so one copy from ``host_inputs()`` refills them.  ``capture`` records
+a step in a CUDA graph, the way a serving loop replays a steady decode step
+without paying the host cost of each call again.
 """
 from __future__ import annotations
 
