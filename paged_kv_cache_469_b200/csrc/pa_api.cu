@@ -41,6 +41,19 @@ static int part_tokens_for_step(long total_unit_keys, int wave_ctas, int floor_t
   return (int)part;
 }
 
+int device_sm_count() {
+  static std::atomic<int> n[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int v = n[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return 148;
+    n[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
 WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_seq_len) {
   WorkspaceLayout w{};

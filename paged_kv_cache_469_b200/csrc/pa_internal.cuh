@@ -30,6 +30,9 @@ inline cudaError_t raise_smem_limit(Kernel kernel, int bytes, std::atomic<int> (
   return e;
 }
 
+// SMs of the current device (looked up once per device; 148 if the query fails)
+int device_sm_count();
+
 constexpr int kBlockSize = 16;       // tokens per cache block (the pages' default)
 constexpr int kDecodeRows = 16;      // query rows per kv-head one decode CTA holds (MMA M)
 // A decode-class sequence has at most kDecodeMaxRows query rows per kv-head

@@ -184,15 +184,6 @@ plan_step_kernel(const int32_t* __restrict__ free_queue, int queue_len, int32_t*
   }
 }
 
-int sm_count_plan() {
-  static int n[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!n[dev]) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
-  return n[dev] > 0 ? n[dev] : 148;
-}
-
 }  // namespace
 
 size_t plan_step_smem(int num_seqs) { return (size_t)(3 * num_seqs + 2) * sizeof(int); }
@@ -204,7 +195,7 @@ cudaError_t launch_plan_step(const int32_t* free_queue, int queue_len, int32_t* 
                              int64_t* slot_mapping, int max_tokens, cudaStream_t stream) {
   // enough CTAs that each writes at most about two slots per thread
   const long long work = max((long long)max_tokens, 1LL);
-  const int grid = (int)min((long long)sm_count_plan(),
+  const int grid = (int)min((long long)device_sm_count(),
                             (work + 2 * kPlanThreads - 1) / (2 * kPlanThreads));
   const int smem = (int)plan_step_smem(num_seqs);
   if (smem > 48 * 1024) {

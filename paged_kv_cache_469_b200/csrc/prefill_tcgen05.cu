@@ -819,15 +819,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  static int n[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!n[dev]) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
-  return n[dev] > 0 ? n[dev] : 148;
-}
-
 // The work list of prefill_plan_kernel, built on the host from its copies of
 // the step's lengths: the same items, heaviest first.  False when there are
 // more items than a kernel parameter holds.
@@ -918,7 +909,7 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items,
                                    : (int)min((long)p.max_items,
                                               (long)p.num_seqs * ((max_query_len + QT - 1) / QT) *
                                                   p.num_q_heads);
-  const int grid = max(1, min(sm_count(), upper));
+  const int grid = max(1, min(device_sm_count(), upper));
   auto kernel = prefill_tcgen05_kernel<D>;
   const int smem = PrefillLayout<D>::total;
   static std::atomic<int> smem_done[64];
