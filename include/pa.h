@@ -253,7 +253,11 @@ int pa_attention_varlen_static_scratch(
  * the blocks a request lacks from the front of free_block_queue into the
  * request's block list, requests in order; the step's sequences form one
  * super-sequence; a token at position p is stored in slot
- * block_table[p / 16] * 16 + p % 16.  (Step 2 of allocate_slots, preempting
+ * block_table[p / 16] * 16 + p % 16.  Page "【ITニュース解説】Inside vLLM: Anatomy
+ * of a High-Throughput LLM Inference System", its paragraph on Paging
+ * Attention: blocks are handed out as the model produces new tokens, only as
+ * many as are needed, so a running request grows by whole blocks step by
+ * step.  (Step 2 of allocate_slots, preempting
  * requests when the pool runs dry, is scheduler policy: here a step that does
  * not fit is refused, see the status bits.)
  *

@@ -150,7 +150,10 @@ int oracle_slot_mapping(const int32_t* block_tables, int max_blocks_per_seq,
   return 0;
 }
 
-/* One scheduler step of block planning for a running batch.  Sequence s
+/* One scheduler step of block planning for a running batch (page
+ * "【ITニュース解説】Inside vLLM: Anatomy of a High-Throughput LLM Inference
+ * System", its paragraph on Paging Attention: blocks are handed out as new
+ * tokens are produced, only as many as needed).  Sequence s
  * holds the blocks of its first num_computed[s] tokens (the first
  * blocks_needed(num_computed[s]) entries of its row) and schedules
  * query_lens[s] new tokens.  allocate_slots, sequences in order: each takes
