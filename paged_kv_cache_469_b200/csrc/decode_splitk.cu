@@ -33,8 +33,8 @@
 // Split-K.  A CTA reduces its warps' (max, sum, O) in shared memory.  A
 // sequence that fits one partition writes its output directly; otherwise each
 // partition stores its fp32 partial in the workspace and bumps a per
-// (sequence, kv-head) counter; the CTA that arrives last merges all partials
-// and resets the counter.  No CTA ever waits for another.
+// (sequence, kv-head, row group) counter; the CTA that arrives last merges
+// all partials and resets the counter.  No CTA ever waits for another.
 //
 // The kernel is launched as a programmatic dependent of whatever precedes it
 // on the stream (typically the cache write), so its launch overlaps that
