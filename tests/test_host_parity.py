@@ -52,3 +52,34 @@ def test_worked_example_and_pool_exhaustion():
     assert pool.allocate_slots("a", 32) == []  # still fits in 2 blocks
     with pytest.raises(PoolExhausted):
         pool.allocate_slots("b", 33)
+
+
+@pytest.mark.parametrize("seed", [3, 4])
+def test_host_pool_across_steps_matches_oracle_plan_step(seed, oracle_lib):
+    """A BlockPool kept across scheduler steps (each step: allocate_slots of
+    every sequence's new length, then the table, slots and offsets) gives the
+    oracle's plan_step step for step -- the same steps pa_plan_step runs on
+    the GPU."""
+    from paged_kv_cache_469_b200.block_pool import query_start_loc, slot_mapping
+    from paged_kv_cache_469_b200.inputs import planner_draws
+    S, mb = 30, 96
+    fq, nc, ql = planner_draws(seed, num_seqs=S, num_blocks=5000, max_ctx=600, max_chunk=90,
+                               prefill_frac=0.3, idle_frac=0.1)
+    pool = BlockPool(fq)
+    for s in range(S):
+        pool.allocate_slots(s, int(nc[s]))
+    tables = pool.block_table(range(S), mb)
+    head = len(fq) - len(pool.free_block_queue)
+    rng = np.random.default_rng(seed)
+    for _ in range(5):
+        want = oracle.plan_step(fq, head, tables, nc, ql)
+        for s in range(S):
+            pool.allocate_slots(s, int(nc[s] + ql[s]))
+        tables = pool.block_table(range(S), mb)
+        np.testing.assert_array_equal(tables, want[0])
+        np.testing.assert_array_equal(slot_mapping(tables, nc, ql), want[3])
+        np.testing.assert_array_equal(query_start_loc(ql), want[2])
+        head = len(fq) - len(pool.free_block_queue)
+        assert head == want[4]
+        nc = want[1]
+        ql = np.where(rng.random(S) < 0.2, rng.integers(0, 80, S), 1).astype(np.int32)
