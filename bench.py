@@ -10,14 +10,21 @@ step's attention must read (sum over sequences of seq_len * 2 * Hkv * D * 2 B,
 summed over ranks) divided by the device time of a step (max over ranks).
 Steps run back to back, as in a serving loop, each one a single
 pa_attention_varlen_write_cache call (cache write fused into the decode
-kernel): timed both as one CUDA graph replay per step and as plain calls
-(each launch a programmatic dependent of the previous one); `value` uses the
-faster and `launch` says which.  No step finds its inputs in L2:
-when one step reads less than twice the L2 size, the timed loop rotates over
-that many identical copies of the workload (own pool, own tensors) that
-consecutive reads of one copy are separated by more than twice the L2 size of
-other traffic.  `--impl reference` times the CPU oracle on a bounded sample of
-the same workload instead.
+kernel).  Every timed figure is one replay of one CUDA graph holding exactly
+--steps back-to-back calls (each launch a programmatic dependent of the one
+before), timed with CUDA events on the launching stream, so the number is the
+GPU's time and does not depend on how fast the host issues calls.  No step
+finds its inputs in L2: when one step reads less than twice the L2 size, the
+steps rotate over that many identical copies of the workload (own pool, own
+tensors) that consecutive reads of one copy are separated by more than twice
+the L2 size of other traffic.
+
+The line also carries the mixed prefill + decode step (query tokens/s, and its
+prefill chunks alone against the bf16 peak), the prefix-cached decode step
+(unique and logical KV GB/s), the long-context decode step, the on-GPU step
+planner, and the end-to-end figure from pinned host buffers.
+`--impl reference` times the CPU oracle on a bounded sample of the decode
+workload instead.
 """
 from __future__ import annotations
 
@@ -39,10 +46,12 @@ MIXED_WORKLOAD = "mixed_llama3_8b"
 L2_BYTES = 126 * 1000 * 1000  # B200 L2, for sizing the rotation of workload copies
 MAX_COPIES = 8
 REFERENCE_BUDGET_S = 120.0  # host seconds the --impl reference steps may take in all
-# dram__bytes_read.sum + dram__bytes_write.sum of one decode_splitk_kernel<64,false,4,4,false>
-# launch on this workload, from an ncu --set full capture of that launch; set
-# to None whenever that kernel changes, until it is captured again
-DECODE_TRAFFIC_BYTES = 68_948_736 + 1_102_080
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of DECODE_KERNEL
+# on this workload, from an ncu capture of that launch; None whenever that
+# kernel has changed since it was last captured
+DECODE_TRAFFIC_BYTES = None
+DECODE_KERNEL = "decode_persistent_kernel<64,8,false>"
+KERNELS_PER_DECODE_STEP = 1  # the decode step is one launch (cache write inside the kernel)
 
 
 def kv_bytes(step, seqs=None) -> int:
@@ -269,6 +278,16 @@ def step_bytes(step) -> int:
     return kv_bytes(step) + 2 * int(step.q.size) * elem
 
 
+def unique_kv_bytes(step) -> int:
+    """K+V bytes of the distinct cache tokens a step reads: a shared prefix counts once."""
+    import numpy as np
+    p = int(step.shared_prefix_tokens)
+    lens = step.seq_lens.astype(np.int64)
+    tokens = int(lens.sum()) - p * max(0, step.num_seqs - 1)
+    elem = 4 if step.dtype == "f32" else 2
+    return tokens * 2 * step.num_kv_heads * step.head_dim * elem
+
+
 def copies_for(step) -> int:
     """Copies of the workload to rotate over so that no step finds its inputs in
     L2: enough that the other copies' traffic between two reads of one copy
@@ -277,18 +296,68 @@ def copies_for(step) -> int:
     return int(min(MAX_COPIES, max(1, -(-2 * L2_BYTES // b) + 1))) if b < 2 * L2_BYTES else 1
 
 
-def timed_loop(fns, stream, steps: int) -> float:
-    """Mean device ms per call over `steps` back-to-back calls of fns[i % len(fns)]
-    (CUDA events on the launching stream around the whole loop)."""
+def _upload(g) -> None:
+    """Upload an instantiated graph to the device before it is timed, so that
+    the first timed replay does not include the upload."""
+    import ctypes
+    import torch
+    try:
+        cu = ctypes.CDLL("libcuda.so.1")
+        cu.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        cu.cuGraphUpload.restype = ctypes.c_int
+        rc = cu.cuGraphUpload(ctypes.c_void_p(g.raw_cuda_graph_exec()),
+                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        torch.cuda.synchronize()
+        if rc != 0:
+            raise RuntimeError(f"cuGraphUpload returned {rc}")
+    except (OSError, AttributeError):
+        pass
+
+
+def capture_steps(calls, k: int):
+    """One CUDA graph of k back-to-back calls, calls[i % len(calls)]() for i < k.
+    Each call is made once outside the capture first (one-time set-up)."""
+    import torch
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(k):
+            calls[i % len(calls)]()
+    _upload(g)
+    return g
+
+
+def time_graph(g, stream) -> float:
+    """Device ms of one replay of g (CUDA events on the launching stream,
+    synchronised on both sides)."""
     import torch
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
     a.record(stream)
-    for i in range(steps):
-        fns[i % len(fns)]()
+    g.replay()
     b.record(stream)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps
+    return a.elapsed_time(b)
+
+
+def timed_steps(calls, args, stream, world, clocks) -> float:
+    """Mean device ms per call: args.warmup untimed calls (one graph), then one
+    replay of a graph of exactly args.steps back-to-back calls, timed; the max
+    over ranks."""
+    import torch
+    warm = capture_steps(calls, args.warmup)
+    warm.replay()
+    g = capture_steps(calls, args.steps)
+    torch.cuda.synchronize()
+    barrier(world)
+    with clocks.window() if clocks else _nullctx():
+        ms = time_graph(g, stream)
+    barrier(world)
+    del g, warm
+    return max_over_ranks(ms / args.steps, world)
 
 
 def prefill_flops(step) -> int:
@@ -302,53 +371,43 @@ def prefill_flops(step) -> int:
     return 4 * step.head_dim * step.num_q_heads * pairs
 
 
+def _free(*objs):
+    import torch
+    del objs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
 def bench_mixed(args, dev, stream, world, clocks):
     """Mixed prefill + decode step (Llama-3-8B attention shape): query tokens/s,
     plus the prefill chunks alone against the bf16 tensor peak."""
-    import torch
     from paged_kv_cache_469_b200.inputs import prefill_part, workload
     from paged_kv_cache_469_b200.step import DeviceStep
     step = workload(MIXED_WORKLOAD)
-    n = min(args.steps, 200)
     dss = [DeviceStep(step, device=str(dev)) for _ in range(copies_for(step))]
-    graphs = [d.capture("fused") for d in dss]
-    for i in range(args.warmup):
-        graphs[i % len(dss)].replay()
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    with clocks.window() if clocks else _nullctx():
-        step_ms = timed_loop([g.replay for g in graphs], stream, n)
-    barrier(world)
-    step_ms = max_over_ranks(step_ms, world)
+    copies = len(dss)
+    step_ms = timed_steps([d.run_fused for d in dss], args, stream, world, clocks)
     tokens = sum_over_ranks(step.num_tokens, world)
     g = step.num_q_heads // step.num_kv_heads
     kv_dec = int(sum(L for L, q in zip(step.seq_lens.tolist(), step.query_lens.tolist())
                      if q * g <= 64)) * 2 * step.num_kv_heads * step.head_dim * 2
-    copies = len(dss)
-    del dss, graphs
-    torch.cuda.empty_cache()
+    _free(*dss)
+    del dss
     # the same step's prefill chunks alone (same lengths, same shape)
     pre = prefill_part(step)
     dps = [DeviceStep(pre, device=str(dev)) for _ in range(copies_for(pre))]
-    pgraphs = [d.capture("attention") for d in dps]
-    for i in range(args.warmup):
-        pgraphs[i % len(dps)].replay()
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    with clocks.window() if clocks else _nullctx():
-        pre_ms = timed_loop([g.replay for g in pgraphs], stream, n)
-    barrier(world)
-    pre_ms = max_over_ranks(pre_ms, world)
+    pre_ms = timed_steps([d.attention for d in dps], args, stream, world, clocks)
     flops = prefill_flops(pre)
     peaks = load_peaks()
     tflops = flops / (pre_ms / 1e3) / 1e12
     pre_copies = len(dps)
-    del dps, pgraphs
-    torch.cuda.empty_cache()
+    _free(*dps)
+    del dps
     return {"workload": MIXED_WORKLOAD, "value": round(tokens / (step_ms / 1e3), 1),
-            "unit": "query tokens/s", "ms_per_step": round(step_ms, 4), "steps": n,
+            "unit": "query tokens/s", "ms_per_step": round(step_ms, 4), "steps": args.steps,
             "query_tokens_per_step_per_gpu": step.num_tokens,
             "decode_kv_bytes_per_step_per_gpu": kv_dec, "copies_rotated": copies,
+            "launch": "one CUDA graph of --steps back-to-back pa_attention_varlen_write_cache calls",
             "prefill_only": {"ms": round(pre_ms, 4), "gflop": round(flops / 1e9, 3),
                              "tflops": round(tflops, 1),
                              "frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
@@ -357,6 +416,35 @@ def bench_mixed(args, dev, stream, world, clocks):
                              "peak_source": peaks["source"], "copies_rotated": pre_copies,
                              "kernels": ("prefill_tcgen05_kernel<128> (work list from the "
                                          "host copies of the step's lengths)")}}
+
+
+def bench_decode_workload(name, args, dev, stream, world, clocks):
+    """A decode-class workload's step (cache write of the new tokens + attention,
+    one pa_attention_varlen_write_cache call): KV GB/s against the HBM peak."""
+    from paged_kv_cache_469_b200.inputs import workload
+    from paged_kv_cache_469_b200.step import DeviceStep
+    step = workload(name)
+    dss = [DeviceStep(step, device=str(dev)) for _ in range(copies_for(step))]
+    copies = len(dss)
+    ms = timed_steps([d.run_fused for d in dss], args, stream, world, clocks)
+    _free(*dss)
+    del dss
+    peaks = load_peaks()
+    logical = sum_over_ranks(kv_bytes(step), world)
+    unique = sum_over_ranks(unique_kv_bytes(step), world)
+    gbs = unique / (ms / 1e3) / 1e9
+    rec = {"workload": name, "unit": "GB/s", "ms_per_step": round(ms, 4), "steps": args.steps,
+           "num_seqs": step.num_seqs, "context_tokens": int(step.seq_lens.sum()),
+           "value": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4),
+           "peak_source": f"{peaks['source']} HBM copy bandwidth",
+           "kv_bytes_per_step_per_gpu": unique_kv_bytes(step), "copies_rotated": copies,
+           "launch": "one CUDA graph of --steps back-to-back pa_attention_varlen_write_cache calls"}
+    if step.shared_prefix_tokens:
+        rec["bytes"] = ("unique: the shared prefix's blocks counted once (the roofline "
+                        "figure); logical: every sequence's keys")
+        rec["logical_kv_bytes_per_step_per_gpu"] = kv_bytes(step)
+        rec["logical_gbs"] = round(logical / (ms / 1e3) / 1e9, 1)
+    return rec
 
 
 def bench_planner(args, dev, stream) -> dict:
@@ -400,7 +488,7 @@ def bench_planner(args, dev, stream) -> dict:
     slots = torch.empty(int(ql.sum()), dtype=torch.int64, device=dev)
 
     def call():
-        lib.plan_step(fq, state, nc_t, ql_t, tables, seq_lens, qsl, slots, stream=stream)
+        lib.plan_step(fq, state, nc_t, ql_t, tables, seq_lens, qsl, slots)
 
     call()
     torch.cuda.synchronize(dev)
@@ -411,15 +499,17 @@ def bench_planner(args, dev, stream) -> dict:
             np.array_equal(seq_lens.cpu().numpy(), nc + ql) and
             state.cpu().tolist()[:3] == [head0 + per_call, 0, 0]):
         raise RuntimeError("pa_plan_step and the host planner disagree")
-    # every call repeats the step (same counts, the next blocks of the queue)
+    # every call repeats the step (same counts, the next blocks of the queue);
+    # the queue must hold the blocks of every call, warm-up included
     left = len(step.free_queue) - head0 - per_call
-    n = int(max(1, min(args.steps, left // max(1, per_call) - args.warmup)))
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize(dev)
-    dev_us = timed_loop([call], stream, n) * 1e3
+    n = int(max(1, min(args.steps, left // max(1, per_call) - 2 * args.warmup - 2)))
+    warm = capture_steps([call], args.warmup)
+    warm.replay()
+    g = capture_steps([call], n)
+    dev_us = time_graph(g, stream) * 1e3 / n
     if state[1].item() != 0:
         raise RuntimeError("pa_plan_step refused a timed call")
+    del g, warm
 
     def pinned_like(a):
         return torch.from_numpy(np.empty_like(a)).pin_memory()
@@ -449,7 +539,7 @@ def bench_planner(args, dev, stream) -> dict:
     return {"workload": WORKLOAD, "num_seqs": S, "new_tokens": int(ql.sum()),
             "blocks_taken_per_call": per_call,
             "device_us_per_call": round(dev_us, 3), "calls": n,
-            "device_timing": "back-to-back pa_plan_step calls, CUDA events around the loop",
+            "device_timing": "one CUDA graph of back-to-back pa_plan_step calls, CUDA events",
             "host_us_per_step": round(statistics.median(host_us), 1),
             "host_path": ("BlockPool.allocate_slots per sequence, block_table, slot_mapping, "
                           "query_start_loc, four pinned copies to the device, stream sync "
@@ -457,8 +547,135 @@ def bench_planner(args, dev, stream) -> dict:
             "equal_outputs": True}
 
 
-def bench_ours(args) -> None:
+def bench_device_loop(args, dev, stream, world, clocks) -> dict:
+    """The serving loop planned on the GPU: every step is pa_plan_step (one
+    token more per sequence), pa_attention_varlen_write_cache without host
+    copies (its decode work listed on the device) and the new lengths copied
+    into num_computed, for the decode workload's 64 sequences, starting from
+    its contexts.  --steps such steps are captured as one CUDA graph, rotating
+    over the same copies of the workload as the main leg, and timed as one
+    replay.  Query tokens/s (one per sequence and step), and KV GB/s on the
+    keys the steps actually read (the sequences grow by one token per step)."""
     import numpy as np
+    import torch
+    from paged_kv_cache_469_b200 import lib
+    from paged_kv_cache_469_b200.inputs import workload
+    from paged_kv_cache_469_b200.step import DeviceStep
+    step = workload(WORKLOAD)
+    n = copies_for(step)
+    per_copy = -(-(args.steps + args.warmup) // n) + 4  # steps each copy takes at most
+    bound = int(step.seq_lens.max()) + per_copy
+    loops = []
+    for _ in range(n):
+        d = DeviceStep(step, device=str(dev), max_blocks_per_seq=-(-bound // 16))
+        S = step.num_seqs
+        st = {"d": d,
+              "fq": torch.from_numpy(step.free_queue).to(dev),
+              "state": lib.new_planner_state(d.plan.blocks_taken, device=dev),
+              "num_computed": d.seq_lens.clone(),
+              "query_lens": torch.ones(S, dtype=torch.int32, device=dev),
+              "seq_lens": torch.empty(S, dtype=torch.int32, device=dev),
+              "qsl": torch.empty(S + 1, dtype=torch.int32, device=dev),
+              "slots": torch.empty(S, dtype=torch.int64, device=dev),
+              "ws": lib.new_workspace(S, step.num_q_heads, step.num_kv_heads, step.head_dim,
+                                      bound, device=dev)}
+        loops.append(st)
+
+    def call_for(st):
+        d = st["d"]
+
+        def call():
+            lib.plan_step(st["fq"], st["state"], st["num_computed"], st["query_lens"],
+                          d.block_tables, st["seq_lens"], st["qsl"], st["slots"])
+            lib.attention_varlen_write_cache(
+                d.out, d.q, d.k_new, d.v_new, d.k_cache, d.v_cache, st["slots"], d.block_tables,
+                st["seq_lens"], st["qsl"], max_query_len=1, max_seq_len=bound,
+                scale=step.scale, workspace=st["ws"])
+            st["num_computed"].copy_(st["seq_lens"])
+        return call
+
+    calls = [call_for(st) for st in loops]
+    # every call (the set-up call of capture_steps and the warm-up included)
+    # advances its copy by one token per sequence
+    ms = timed_steps(calls, args, stream, world, clocks)
+    if any(int(st["state"][1].item()) != 0 for st in loops):
+        raise RuntimeError("pa_plan_step refused a step of the device-planned loop")
+    # keys read by the timed steps: copy c's k-th step reads the contexts + k + 1
+    lens0 = step.seq_lens.astype(np.int64)
+    done = [0] * n
+    for c in range(n):  # set-up calls: one per copy per captured graph, plus the warm-up
+        done[c] = 2
+    for i in range(args.warmup):
+        done[i % n] += 1
+    keys = 0
+    for i in range(args.steps):
+        c = i % n
+        keys += int((lens0 + done[c] + 1).sum())
+        done[c] += 1
+    kv = keys * 2 * step.num_kv_heads * step.head_dim * 2
+    tokens = sum_over_ranks(step.num_seqs, world)
+    del loops, calls
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return {"workload": WORKLOAD, "num_seqs": step.num_seqs, "steps": args.steps,
+            "copies_rotated": n, "ms_per_step": round(ms, 5),
+            "value": round(tokens / (ms / 1e3), 1), "unit": "query tokens/s",
+            "kv_gbs": round(sum_over_ranks(kv, world) / args.steps / (ms / 1e3) / 1e9, 1),
+            "launch": ("one CUDA graph of --steps steps, each pa_plan_step + "
+                       "pa_attention_varlen_write_cache (no host copies) + a copy of the new "
+                       "lengths; no host work between steps")}
+
+
+def capture_e2e(dss, host_ins, host_out, k: int):
+    """One CUDA graph of k steps end to end: step i copies its packed inputs in
+    from pinned host memory (copy stream), runs pa_attention_varlen_write_cache
+    (launching stream) and copies its output back (second copy stream).  At
+    most two steps are in flight: step i's input copy waits for step i-2's
+    kernel, and step i's kernel for step i-2's output copy, so that step i+1's
+    copy in and step i-1's copy out overlap step i's kernel while no buffer is
+    overwritten before it has been read."""
+    import torch
+    c = len(dss)
+    depth = min(2, c)
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+    for d, h in zip(dss, host_ins):  # one eager step per copy (one-time set-up)
+        d.inputs.copy_(h, non_blocking=True)
+        d.run_fused()
+        host_out.copy_(d.out.view(torch.int16), non_blocking=True)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cap = torch.cuda.current_stream()
+        start = torch.cuda.Event()
+        start.record(cap)
+        k_done, o_done = [], []
+        for i in range(k):
+            d = dss[i % c]
+            cin.wait_event(k_done[i - depth] if i >= depth else start)
+            with torch.cuda.stream(cin):
+                d.inputs.copy_(host_ins[i % c], non_blocking=True)
+            e_in = torch.cuda.Event()
+            e_in.record(cin)
+            cap.wait_event(e_in)
+            if i >= depth:
+                cap.wait_event(o_done[i - depth])
+            d.run_fused()
+            e_k = torch.cuda.Event()
+            e_k.record(cap)
+            k_done.append(e_k)
+            cout.wait_event(e_k)
+            with torch.cuda.stream(cout):
+                host_out.copy_(d.out.view(torch.int16), non_blocking=True)
+            e_o = torch.cuda.Event()
+            e_o.record(cout)
+            o_done.append(e_o)
+        cap.wait_stream(cin)
+        cap.wait_stream(cout)
+    _upload(g)
+    return g
+
+
+def bench_ours(args) -> None:
     import torch
 
     from paged_kv_cache_469_b200 import lib
@@ -472,90 +689,45 @@ def bench_ours(args) -> None:
     stream = torch.cuda.current_stream(dev)
     dss = [DeviceStep(step, device=str(dev)) for _ in range(copies_for(step))]
     copies = len(dss)
-
-    # ---- device-resident steps, back to back over the rotating copies: one
-    # CUDA graph replay per step (and, for reference, plain stream launches)
-    step_graphs = [d.capture("fused") for d in dss]
-    attn_graphs = [d.capture("attention") for d in dss]
-    for i in range(args.warmup):
-        step_graphs[i % copies].replay()
-        dss[i % copies].run_fused()
-    torch.cuda.synchronize(dev)
     clocks = ClockSampler(local) if rank == 0 or world > 1 else None
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with clocks.window() if clocks else _nullctx():
-        step_ms = timed_loop([g.replay for g in step_graphs], stream, args.steps)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    # the attention call alone (the roofline's kernel): back-to-back stream
-    # launches, each a programmatic dependent of the one before, so that the
-    # interval is the kernel's own time (a one-kernel graph per call would add
-    # its launch gap)
-    with clocks.window() if clocks else _nullctx():
-        attn_ms = timed_loop([d.attention for d in dss], stream, args.steps)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with clocks.window() if clocks else _nullctx():
-        attn_graph_ms = timed_loop([g.replay for g in attn_graphs], stream, args.steps)
-    barrier(world)
-    attn_graph_ms = max_over_ranks(attn_graph_ms, world)
-    torch.cuda.synchronize(dev)
-    with clocks.window() if clocks else _nullctx():
-        stream_step_ms = timed_loop([d.run_fused for d in dss], stream, args.steps)
-    barrier(world)
-    stream_step_ms = max_over_ranks(stream_step_ms, world)
-    step_ms_max = max_over_ranks(step_ms, world)
-    graph_step_ms = step_ms_max
-    # the headline is the faster of the two ways to run the step: graph replays
-    # (one per step) or plain back-to-back calls (each launch a programmatic
-    # dependent of the previous one, which graph replays cannot be)
-    launch = ("one CUDA graph replay per step of pa_attention_varlen_write_cache "
-              "(cache write fused into the decode kernel)")
-    if stream_step_ms < step_ms_max:
-        step_ms_max = stream_step_ms
-        launch = ("back-to-back pa_attention_varlen_write_cache calls, one per step "
-                  "(cache write fused into the decode kernel; each launch a programmatic "
-                  "dependent of the previous step's)")
-    attn_ms_max = max_over_ranks(attn_ms, world)
+
+    # ---- device-resident steps: one CUDA graph of --steps back-to-back
+    # pa_attention_varlen_write_cache calls over the rotating copies, timed
+    # as one replay (each launch a programmatic dependent of the previous one)
+    step_ms = timed_steps([d.run_fused for d in dss], args, stream, world, clocks)
+    # the attention call alone (the roofline's kernel), the same way
+    attn_ms = timed_steps([d.attention for d in dss], args, stream, world, clocks)
     bytes_rank = kv_bytes(step)
     bytes_all = sum_over_ranks(bytes_rank, world)
-    value = bytes_all / (step_ms_max / 1e3) / 1e9
+    value = bytes_all / (step_ms / 1e3) / 1e9
 
     # ---- end to end through the public API from pinned host buffers: every step
     # copies its inputs in (one copy: the step's inputs are packed into one
     # buffer on both sides), runs, and copies its output back
-    ds0 = dss[0]
     host_ins = [d.host_inputs() for d in dss]
-    host_out = torch.empty(ds0.out.shape, dtype=torch.int16).pin_memory()
+    host_out = torch.empty(dss[0].out.shape, dtype=torch.int16).pin_memory()
     h2d = host_ins[0].numel()
     d2h = host_out.numel() * host_out.element_size()
-
-    def e2e_graph(r):
-        d, hin = dss[r], host_ins[r]
-
-        def copies_in():
-            d.inputs.copy_(hin, non_blocking=True)
-
-        def copy_out():
-            host_out.copy_(d.out.view(torch.int16), non_blocking=True)
-        return d.capture("fused", prologue=copies_in, epilogue=copy_out)
-
-    e2e_graphs = [e2e_graph(r) for r in range(copies)]
-    for i in range(args.warmup):
-        e2e_graphs[i % copies].replay()
-    torch.cuda.synchronize(dev)
+    warm = capture_e2e(dss, host_ins, host_out, args.warmup)
+    warm.replay()
+    g = capture_e2e(dss, host_ins, host_out, args.steps)
     barrier(world)
-    torch.cuda.synchronize(dev)
     with clocks.window() if clocks else _nullctx():
-        e2e_ms = timed_loop([g.replay for g in e2e_graphs], stream, args.steps)
+        e2e_ms = time_graph(g, stream) / args.steps
     barrier(world)
     e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_value = bytes_all / (e2e_ms / 1e3) / 1e9
-    del dss, host_ins, ds0, step_graphs, attn_graphs, e2e_graphs
-    torch.cuda.empty_cache()
+    del g, warm, host_ins
+    _free(*dss)
+    del dss
     mixed = None if args.no_mixed else bench_mixed(args, dev, stream, world, clocks)
+    prefix = (None if args.no_decode_configs else
+              bench_decode_workload("prefix_decode_llama3_8b", args, dev, stream, world, clocks))
+    long_ = (None if args.no_decode_configs else
+             bench_decode_workload("long_decode_llama3_8b", args, dev, stream, world, clocks))
     planner = None if args.no_planner or rank != 0 else bench_planner(args, dev, stream)
+    device_loop = (None if args.no_planner else
+                   bench_device_loop(args, dev, stream, world, clocks))
     clk = clocks.stop() if clocks else None
 
     if rank != 0:
@@ -565,11 +737,14 @@ def bench_ours(args) -> None:
         return
 
     peaks = load_peaks()
-    achieved = bytes_rank / (attn_ms_max / 1e3) / 1e9
+    achieved = bytes_rank / (attn_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": DECODE_TRAFFIC_BYTES, "traffic_unit": "bytes per launch (ncu)",
-                "kernel": "decode_splitk_kernel<64,false,4,4,false> (attention call without the fused cache write)",
+                "traffic": DECODE_TRAFFIC_BYTES,
+                "traffic_unit": "dram bytes read + written per launch (ncu)",
+                "kernel": DECODE_KERNEL + " (attention call without the fused cache write)",
+                "timing": ("one CUDA graph of --steps back-to-back attention calls over the "
+                           "rotating copies, CUDA events around one replay"),
                 "peak_source": f"{peaks['source']} HBM copy bandwidth (burst)",
                 "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)}
     cpu = None
@@ -584,8 +759,9 @@ def bench_ours(args) -> None:
                                  "sample": f"first {n1} sequences, {passes1} passes, "
                                            f"{dt1:.1f} s"},
                "cpu_model": cpu_model()}
+    launches = args.steps * KERNELS_PER_DECODE_STEP
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "num_seqs": step.num_seqs,
@@ -596,16 +772,20 @@ def bench_ours(args) -> None:
                              f"copies of the workload, {copies * step_bytes(step) / 1e6:.0f} MB "
                              f"touched per rotation)",
                        "parallelism": f"{world} independent replicas"},
-            "attention_ms": round(attn_ms_max, 5),
-            "launch": launch,
-            "graph_replay_ms_per_step": round(graph_step_ms, 5),
-            "stream_launch_ms_per_step": round(stream_step_ms, 5),
-            "attention_graph_replay_ms": round(attn_graph_ms, 5),
-            "gpu_launches": args.steps,
+            "attention_ms": round(attn_ms, 5),
+            "launch": ("one CUDA graph of --steps back-to-back pa_attention_varlen_write_cache "
+                       "calls (cache write fused into the decode kernel; each launch a "
+                       "programmatic dependent of the previous step's), timed as one replay"),
+            "gpu_launches": launches,
             "mixed_step": mixed,
+            "prefix_decode": prefix,
+            "long_decode": long_,
             "plan_step": planner,
-            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 4),
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "device_planned_loop": device_loop,
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "overlap": ("copy in, kernel and copy out on three streams, at most two "
+                                "steps in flight")},
             "roofline": roofline, "cpu_baseline": cpu, "clocks": clk}
     print(json.dumps(line), flush=True)
     if world > 1:
@@ -624,6 +804,8 @@ def main(argv=None) -> None:
                     help="skip the mixed prefill+decode leg (Llama-3-8B shape)")
     ap.add_argument("--no-planner", action="store_true",
                     help="skip the on-GPU step planner measurement")
+    ap.add_argument("--no-decode-configs", action="store_true",
+                    help="skip the prefix-cached and long-context decode legs")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

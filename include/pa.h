@@ -17,9 +17,12 @@
  *
  * Conventions of every call:
  *   - Every tensor pointer is DEVICE memory owned by the caller, contiguous,
- *     row-major, 16-byte aligned.  The library allocates nothing and keeps no
- *     data between calls; the caller's workspace holds all scratch.  (It does
- *     remember, per device, the kernel attributes it has already set.)
+ *     row-major, 16-byte aligned.  The library allocates no device memory and
+ *     keeps no data between calls; the caller's workspace holds all scratch.
+ *     (It does remember, per device, the kernel attributes it has already
+ *     set, and, per thread and device, the one side stream and two events it
+ *     creates on the first call that runs a mixed step's two classes of work
+ *     side by side; see pa_attention_varlen.)
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and keeps stream order: each kernel is launched
  *     as a programmatic dependent of the work before it, so its launch may
@@ -92,7 +95,8 @@ int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_ca
  * num_seqs sequences, no sequence longer than max_seq_len tokens: a status
  * word, fp32 split-K partials (running max, sum and unnormalised output per
  * partition of a sequence's keys), one int32 arrival counter per (sequence,
- * kv-head) and the prefill work list.  0 means invalid arguments.
+ * kv-head, 16-row group of query rows; four groups per kv-head) and the
+ * prefill work list.  0 means invalid arguments.
  */
 size_t pa_attention_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                    int head_dim, int max_seq_len);
@@ -160,14 +164,21 @@ int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_s
  *
  * Decode-class sequences (q_len * num_q_heads / num_kv_heads <= 64 query
  * rows per kv-head: single-token decodes and the few-token queries of
- * speculative verification) run the split-K bandwidth-bound kernel, 16 rows
- * per CTA; longer prefill chunks run the tensor-core kernel.  fp32 steps run a CUDA-core kernel.
+ * speculative verification) run the persistent split-K bandwidth-bound kernel
+ * (one CTA per SM, pieces of the sequences' blocks claimed largest first, 16
+ * query rows per unit of work); longer prefill chunks run the tensor-core
+ * kernel.  fp32 steps run a CUDA-core kernel.  Without the host copies, a
+ * one-CTA planning kernel first lists the decode work on the device.  When
+ * the host copies show a bf16 step with both classes of sequences, the call
+ * runs the tensor-core prefill kernel on a side stream of its own, on a share
+ * of the SMs proportional to the prefill work, while the decode kernel
+ * streams on the other SMs; `stream` waits for the side stream before the
+ * call returns, so any work queued on `stream` afterwards sees every output
+ * row.  (The side stream joins a stream capture the same way, as a fork and a
+ * join of the captured graph.)
  * Supported: head_dim in {64, 128}; block_size 16; num_q_heads a multiple of
  * num_kv_heads with at most 16 q-heads per kv-head; dtype f32 or bf16;
- * max_seq_len up to at least 1.5M tokens (a longer bound than the split-K
- * merge can hold returns PA_ERR_UNSUPPORTED); at most 65535 sequences in a
- * bf16 call that may hold decode-class sequences (without the host copies,
- * every bf16 call may), else PA_ERR_UNSUPPORTED.
+ * max_seq_len up to 6.2M tokens (a longer bound returns PA_ERR_UNSUPPORTED).
  */
 int pa_attention_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
                         const int32_t* block_tables, int max_blocks_per_seq,
@@ -192,7 +203,9 @@ int pa_attention_varlen(void* out, const void* q, const void* k_cache, const voi
  * When every sequence of the step is decode-class (bf16), the decode kernel
  * writes the rows itself: each CTA first stores the new tokens that fall in
  * its own range of its sequence's keys, then reads them back through the
- * block table.  One launch instead of two.  This requires the usual layout of
+ * block table.  One launch instead of two.  (When a sequence's query rows
+ * span several 16-row groups, each group's CTA stores the same bytes to the
+ * same slots; identical concurrent stores, so every read sees the new row.)  This requires the usual layout of
  * a step: a token's slot is the slot of its own position in its own
  * sequence's block table (block_tables[s][pos / 16] * 16 + pos % 16), and no
  * other sequence of the step reads that slot.  Otherwise (prefill chunks, or
@@ -228,12 +241,21 @@ int pa_attention_varlen_write_cache(
  *
  *   - The first call on each device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address belongs to the CUDA context current at that call: a call
+ *     under another context of the same device (after cudaDeviceReset, or one
+ *     made current through the driver API) looks it up again, which must
+ *     also happen outside a stream capture.
  *   - Every call, on every stream, shares the one array and it keeps the last
  *     call's contents: each call clears the parts that must start at zero.
  *     Calls that can overlap on the GPU (other streams, other threads) race
  *     on the array: serialise them.
  *   - A kernel's status word (see pa_workspace_status) lives in this array
- *     too and is cleared by the next call.
+ *     too and is cleared by the next call.  The caller has no workspace
+ *     pointer to read it through, so a kernel that gave up on one of its
+ *     time-bounded waits (a library bug or a GPU fault, never an input) is
+ *     not reported by this entry point.  Callers that must see that status
+ *     use pa_attention_varlen with a workspace of their own.
+ *   - fp32 steps use no scratch: they are never refused for size.
  */
 #define PA_STATIC_SCRATCH_BYTES (16u << 20)
 int pa_attention_varlen_static_scratch(
@@ -281,8 +303,13 @@ int pa_attention_varlen_static_scratch(
  *                   the call, must be 0 between calls, [3] unused.  Zero it
  *                   once, then set [0] to where the queue's free part starts.
  *   num_computed,
- *   query_lens      int32 [num_seqs] (device; e.g. the previous step's
- *                   seq_lens as num_computed)
+ *   query_lens      int32 [num_seqs] (device; e.g. a copy of the previous
+ *                   step's seq_lens as num_computed).  Neither may share
+ *                   memory with seq_lens, query_start_loc or slot_mapping:
+ *                   the CTAs of one launch read both inputs in full while
+ *                   others already write the outputs, so an aliased buffer
+ *                   would be read half updated.  Such a call returns
+ *                   PA_ERR_INVALID before anything is launched.
  *   block_tables    int32 [num_seqs][max_blocks_per_seq], updated in place
  *   seq_lens        int32 [num_seqs] (written)
  *   query_start_loc int32 [num_seqs + 1] (written)

@@ -1,0 +1,989 @@
+// decode_persistent.cu -- bandwidth-bound paged attention for decode-class
+// sequences, as one persistent grid.
+//
+// Page "LLM推論エンジンvLLMの内部構造を徹底解説", section "エンジンの中核": a decode
+// step runs the newest token against the KV cache and is bound by memory
+// bandwidth; section "PagedAttentionの仕組み": the keys are read block by
+// block through the sequence's block table.
+//
+// Work.  A unit is one (sequence, kv-head, 16-row group of query rows): all
+// q-heads of the kv-head times the sequence's query tokens, up to 64 rows, cut
+// into 16-row groups (a single-token decode with up to 16 q-heads per kv-head
+// is one group, so every K/V byte is read from HBM once per kv-head).  A unit's
+// nblk cache blocks are cut into pieces of P blocks (the last one shorter).
+// The pieces of a launch form one list, largest first (every full piece, then
+// the shorter last pieces by falling size), so that the work still left at the
+// end of the launch is the finest.  P is chosen per launch from the step's
+// total blocks so that every CTA gets a few pieces.
+//
+// Grid.  One CTA per SM (its shared memory holds the streaming rings), each
+// running until the list is exhausted.  CTA b starts with piece b and then
+// claims further pieces from a global counter, one piece ahead of the one it
+// computes, so faster SMs take more pieces.  Inside a CTA:
+//
+//   scheduler warp (the last warp)  claims a piece, copies its block ids and
+//       its query rows into a shared-memory piece slot (two slots: piece p
+//       lives in slot p % 2), writes the step's new K/V rows of the piece into
+//       the cache first when the call asks for it, and publishes the slot.
+//   compute warps 0 .. kWarps-1     warp w takes blocks w, w + kWarps, ... of
+//       every piece.  It streams them through a private ring of kStages
+//       shared-memory stages (K tile + V tile of one (block, kv-head)) with
+//       16-byte cp.async copies, up to kStages blocks in flight, and
+//       the ring runs on from one piece into the next without draining.  Per
+//       16-token block:
+//         S[16 rows x 16 keys] = Q . K^T     mma.m16n8k16 (two per 16 dims of D)
+//         online softmax (fp32 running max and sum, exp2 with log2(e) folded in)
+//         O[16 rows x D]      += P . V       D/8 mma.m16n8k16
+//   piece merge  when a warp has computed its last block of a piece it puts
+//       its (max, sum, O) in a shared merge slot; the last warp to arrive
+//       merges them and writes the piece's result: the output rows when the
+//       piece is the whole unit, else an fp32 partial in the workspace plus an
+//       arrival count per unit, the last arriving piece merging all partials
+//       of its unit into the output.  No CTA ever waits for another.
+//
+// The dot product's D axis is permuted identically on Q and K so that every
+// lane's B-operand words are 8 consecutive bf16 of one key row, and the
+// output's D axis is permuted so that every lane's V words are 8 consecutive
+// bf16 of one key row (undone when the output is stored).  The 16-byte chunks
+// of every tile row are XOR-swizzled on their way into shared memory so that
+// these fragment reads hit distinct banks.
+//
+// Every wait on another warp of the CTA (a piece slot not yet published, the
+// merge slot still in use) is bounded by a time limit; one that runs out sets
+// the workspace status bit and the CTA winds down instead of hanging.  The
+// kernel is launched as a programmatic dependent of whatever precedes it on
+// the stream; it reads nothing before griddepcontrol.wait.
+#include <math.h>
+
+#include "pa_internal.cuh"
+#include "pa_wait.cuh"
+
+namespace pa {
+namespace {
+
+// compute warps and ring stages per CTA, by head_dim and most query rows per
+// unit (shared memory: ring + merge slot + two piece slots, at most 227 KB)
+template <int D, int kMaxRows>
+struct DecodeCfg {
+  static constexpr int kWarps = D == 64 ? 8 : (kMaxRows <= 4 ? 8 : kMaxRows <= 8 ? 7 : 6);
+  static constexpr int kStages = D == 64 ? 4 : 3;
+};
+
+// What the scheduler publishes about one piece.
+struct PieceInfo {
+  int tag;  // CTA-local sequence number of the piece in this slot (-1: none yet)
+  int end;  // 1: the list is exhausted, no piece in this slot
+  int s, kvh, rg, j, nparts;
+  int blk_begin, nb;  // the piece's blocks: blk_begin .. blk_begin + nb - 1 of the sequence
+  int L, ql, q0;
+  int rows, row0;  // this unit's query rows: global rows row0 .. row0 + rows - 1
+};
+
+template <int D, int kMaxRows>
+struct DecodeLayout {
+  static constexpr int kWarps = DecodeCfg<D, kMaxRows>::kWarps;
+  static constexpr int kStages = DecodeCfg<D, kMaxRows>::kStages;
+  static constexpr int kTileBytes = kBlockSize * D * 2;  // one (block, kv-head) tile
+  static constexpr int kStageBytes = 2 * kTileBytes;     // K tile + V tile
+  static constexpr int ring_off = 0;
+  static constexpr int ring_bytes = kWarps * kStages * kStageBytes;
+  // merge slot: per compute warp its rows' max, sum and unnormalised O
+  static constexpr int mm_off = ring_off + ring_bytes;                // [kWarps][kMaxRows]
+  static constexpr int ml_off = mm_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows]
+  static constexpr int mo_off = ml_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows][D]
+  static constexpr int merge_end = mo_off + kWarps * kMaxRows * D * 4;
+  // two piece slots: info, block ids, query rows
+  static constexpr int kInfoBytes = 64;
+  static constexpr int kIdsBytes = kDecodeMaxPieceBlocks * 4;
+  static constexpr int kQBytes = kMaxRows * D * 2;
+  static constexpr int kSlotBytes = kInfoBytes + kIdsBytes + kQBytes;
+  static constexpr int slot_off = (merge_end + 127) / 128 * 128;
+  // per compute warp: (piece, block) of each ring stage
+  static constexpr int meta_off = slot_off + 2 * kSlotBytes;
+  static constexpr int total = meta_off + kWarps * kStages * 8;
+  static_assert(sizeof(PieceInfo) <= kInfoBytes, "piece info");
+  static_assert(kSlotBytes % 16 == 0, "piece slot alignment");
+  static_assert(total <= 227 * 1024, "shared memory of one CTA");
+};
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+// wait until at most `pending` of this thread's newest copy groups are in flight
+template <int kStages>
+__device__ __forceinline__ void cp_async_wait_pending(int pending) {
+  static_assert(kStages <= 5, "cp_async_wait_pending");
+  if (pending <= 0) cp_async_wait<0>();
+  else if (pending == 1) cp_async_wait<1>();
+  else if (pending == 2) cp_async_wait<2>();
+  else if (pending == 3) cp_async_wait<3>();
+  else cp_async_wait<4>();
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// XOR applied to the 16-byte chunk index of tile row `row` (K and V tiles).
+// K rows are read two at a time (rows 2k, 2k+1, chunk 4j..4j+3): flip the
+// half of the 128-byte line on odd rows.  V rows are read four at a time
+// (rows of equal parity), one chunk each: spread them by row bits 1-2.
+__device__ __forceinline__ int k_swz(int row) { return (row & 1) << 2; }
+__device__ __forceinline__ int v_swz(int row) { return row & 6; }
+
+// Output column c (0..7) of n-tile nt sits at dimension 64*(nt/8) + 8*c + nt%8,
+// so a lane owning columns 2*q4, 2*q4+1 of every n-tile owns, per 64-wide
+// half of D, the 16 consecutive dimensions 16*q4 .. 16*q4+15.
+__device__ __forceinline__ int out_dim(int nt, int c) { return 64 * (nt / 8) + 8 * c + (nt % 8); }
+
+// Shared control words of a CTA.
+struct DecodeCtl {
+  int merged;  // CTA-local sequence number of the last piece merged (-1: none)
+  int count;   // compute warps that have put their part of the current piece in the merge slot
+  int abort;   // set by a bounded wait that ran out: every role winds down
+};
+
+// One piece of the list (see DecodeWork): x = sequence, y = ql << 24 | rg << 22
+// | kvh << 12 | part, z = seq_len, w = query_start_loc of the sequence.
+__device__ __forceinline__ int4 load_piece(const AttnParams& p, const DecodeWork& work, int g) {
+  return work.from_ws ? p.ws_pieces[g] : work.items[g];
+}
+
+template <int D, int kMaxRows, bool kWriteCache>
+__global__ void __launch_bounds__((DecodeCfg<D, kMaxRows>::kWarps + 1) * 32, 1)
+decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork work) {
+  using LY = DecodeLayout<D, kMaxRows>;
+  constexpr int kWarps = LY::kWarps;
+  constexpr int kStages = LY::kStages;
+  constexpr bool kRows16 = kMaxRows > 8;
+  constexpr int NJ = D / 32;  // 16-byte K chunks per key row a lane reads
+  constexpr int NV = D / 64;  // 16-byte V chunks per key row a lane reads
+  constexpr int NT = D / 8;   // n-tiles of the P.V product
+  constexpr int NC = D / 16;  // k-chunks of the Q.K^T product
+  constexpr int kChunks = D / 8;                        // 16-byte chunks per tile row
+  constexpr int kCopies = kBlockSize * kChunks / 32;    // 16-byte copies per lane per tile
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ DecodeCtl ctl;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+  auto slot_info = [&](int p_) {
+    return reinterpret_cast<PieceInfo*>(smem + LY::slot_off + (p_ & 1) * LY::kSlotBytes);
+  };
+  auto slot_ids = [&](int p_) {
+    return reinterpret_cast<int*>(smem + LY::slot_off + (p_ & 1) * LY::kSlotBytes +
+                                  LY::kInfoBytes);
+  };
+  auto slot_q = [&](int p_) {  // shared address of the slot's query rows [kMaxRows][D] bf16
+    return sbase + LY::slot_off + (p_ & 1) * LY::kSlotBytes + LY::kInfoBytes + LY::kIdsBytes;
+  };
+  float* msl_m = reinterpret_cast<float*>(smem + LY::mm_off);
+  float* msl_l = reinterpret_cast<float*>(smem + LY::ml_off);
+  float* msl_o = reinterpret_cast<float*>(smem + LY::mo_off);
+  int* meta = reinterpret_cast<int*>(smem + LY::meta_off);  // [kWarps][kStages][2]
+  volatile int* vabort = &ctl.abort;
+  int* status = p.ws_status;
+
+  if (threadIdx.x == 0) {
+    ctl.merged = -1;
+    ctl.count = 0;
+    ctl.abort = 0;
+    slot_info(0)->tag = -1;
+    slot_info(1)->tag = -1;
+  }
+  __syncthreads();
+  // Launched as a programmatic dependent: nothing the preceding kernel may
+  // write is read before this wait; the next kernel may then be launched (it
+  // waits for this grid in the same way).
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  const int G = p.group;
+  const int num_pieces = work.from_ws ? p.ws_header[kWsPieceCount] : work.count;
+  const int P = work.from_ws ? p.ws_header[kWsPieceBlocks] : work.piece_blocks;
+
+  if (warp == kWarps) {
+    // =============================== scheduler ===============================
+    for (int pc = 0;; ++pc) {
+      // slot pc % 2 is free once piece pc - 2 has been merged
+      if (pc >= 2 &&
+          !spin_until([&] { return *(volatile int*)&ctl.merged >= pc - 2; }, vabort, status))
+        break;
+      int g = blockIdx.x;
+      if (pc > 0) {
+        if (lane == 0) g = gridDim.x + atomicAdd(p.ws_header + kWsClaim, 1);
+        g = __shfl_sync(0xffffffffu, g, 0);
+      }
+      PieceInfo* inf = slot_info(pc);
+      if (g >= num_pieces) {
+        if (lane == 0) {
+          inf->end = 1;
+          __threadfence_block();
+          *(volatile int*)&inf->tag = pc;
+        }
+        break;
+      }
+      const int4 it = load_piece(p, work, g);
+      const int s = it.x;
+      const int j = it.y & 0xfff, kvh = (it.y >> 12) & 0x3ff, rg = (it.y >> 22) & 3;
+      const int ql = (it.y >> 24) & 0x7f;
+      const int L = it.z, q0 = it.w;
+      const int nblk = (L + kBlockSize - 1) / kBlockSize;
+      const int nparts = (nblk + P - 1) / P;
+      const int blk_begin = j * P;
+      const int nb = min(P, nblk - blk_begin);
+      const int rows_all = ql * G;
+      const int row0 = kDecodeRows * rg;
+      const int rows = min(kDecodeRows, rows_all - row0);
+      // block ids
+      const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks_per_seq + blk_begin;
+      int* ids = slot_ids(pc);
+      for (int i = lane; i < nb; i += 32) ids[i] = table[i];
+      // query rows (rows past the unit's are zero)
+      {
+        const uint4* qg = (const uint4*)p.q;
+        const uint32_t qs = slot_q(pc);
+        for (int c = lane; c < kMaxRows * kChunks; c += 32) {
+          const int i = c / kChunks, ch = c % kChunks;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (i < rows) {
+            const int gi = row0 + i;
+            const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
+            v = qg[(tok * p.num_q_heads + head) * kChunks + ch];
+          }
+          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(qs + c * 16), "r"(v.x),
+                       "r"(v.y), "r"(v.z), "r"(v.w)
+                       : "memory");
+        }
+      }
+      if constexpr (kWriteCache) {
+        // This step's new tokens of the sequence that fall in the piece's key
+        // range go into their cache slots first (as pa_reshape_and_cache
+        // would); the compute warps read them only after the publication
+        // below.  With several 16-row groups, every row group's piece of the
+        // same (sequence, kv-head, blocks) stores the same bytes to the same
+        // slots, possibly while another CTA reads them: identical concurrent
+        // stores, so every read sees the new row.  No other piece reads
+        // these slots.
+        const int lo = max(L - ql, blk_begin * kBlockSize);
+        const int hi = min(L, (blk_begin + nb) * kBlockSize);
+        if (hi > lo) {
+          const int n = (hi - lo) * kChunks;
+          const int64_t num_slots = (int64_t)p.num_blocks * kBlockSize;
+          const uint4* kn = (const uint4*)p.k_new;
+          const uint4* vn = (const uint4*)p.v_new;
+          uint4* kcw = (uint4*)const_cast<void*>(p.k_cache);
+          uint4* vcw = (uint4*)const_cast<void*>(p.v_cache);
+          for (int i = lane; i < 2 * n; i += 32) {
+            const bool is_v = i >= n;
+            const int ii = is_v ? i - n : i;
+            const int r = ii / kChunks, c = ii % kChunks;
+            const int tok = q0 + (lo - (L - ql)) + r;
+            const int64_t slot = p.slot_mapping[tok];
+            if (slot < 0 || slot >= num_slots) continue;  // padding / out-of-pool slot
+            const int64_t dst =
+                ((slot / kBlockSize * p.num_kv_heads + kvh) * kBlockSize + slot % kBlockSize) *
+                    kChunks + c;
+            const int64_t src = ((int64_t)tok * p.num_kv_heads + kvh) * kChunks + c;
+            if (is_v) vcw[dst] = vn[src];
+            else kcw[dst] = kn[src];
+          }
+          __threadfence();
+        }
+      }
+      if (lane == 0) {
+        inf->end = 0;
+        inf->s = s; inf->kvh = kvh; inf->rg = rg; inf->j = j; inf->nparts = nparts;
+        inf->blk_begin = blk_begin; inf->nb = nb;
+        inf->L = L; inf->ql = ql; inf->q0 = q0;
+        inf->rows = rows; inf->row0 = row0;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        *(volatile int*)&inf->tag = pc;
+      }
+    }
+    // the last CTA to finish claiming resets the claim counter for the next call
+    if (lane == 0) {
+      __threadfence();
+      const int prev = atomicAdd(p.ws_header + kWsDone, 1);
+      if (prev == (int)gridDim.x - 1) {
+        atomicExch(p.ws_header + kWsClaim, 0);
+        atomicExch(p.ws_header + kWsDone, 0);
+      }
+    }
+    return;
+  }
+
+  // ================================ compute warps ================================
+  const int r = lane >> 2, q4 = lane & 3;
+  const char* kc = (const char*)p.k_cache;
+  const char* vc = (const char*)p.v_cache;
+  const int64_t blk_bytes = (int64_t)LY::kTileBytes * p.num_kv_heads;
+  const uint32_t ring = sbase + LY::ring_off + warp * kStages * LY::kStageBytes;
+  int* my_meta = meta + warp * kStages * 2;
+
+  // the piece in slot pc, once published (nullptr before)
+  auto published = [&](int pc) -> const PieceInfo* {
+    const PieceInfo* inf = slot_info(pc);
+    if (*(volatile const int*)&inf->tag != pc) return nullptr;
+    __threadfence_block();
+    return inf;
+  };
+
+  int ip = 0, ii = warp;  // issue cursor: next candidate (piece, block of the piece)
+  bool issue_done = false;
+  int n_issued = 0, n_comp = 0;
+  uint32_t bad = 0;  // bit (stage): that stage's block id was outside the pool
+
+  // Issue the copies of this warp's next block; false when there is none yet
+  // (the next piece is not published and `block` is false) or none at all.
+  auto try_issue = [&](bool block) -> bool {
+    const PieceInfo* inf;
+    while (true) {
+      inf = published(ip);
+      if (!inf) {
+        if (!block) return false;
+        if (!spin_until([&] { return published(ip) != nullptr; }, vabort, status)) {
+          issue_done = true;
+          return false;
+        }
+        inf = published(ip);
+      }
+      if (inf->end) {
+        issue_done = true;
+        return false;
+      }
+      if (ii < inf->nb) break;
+      ++ip;
+      ii = warp;
+    }
+    const int st = n_issued % kStages;
+    int id = slot_ids(ip)[ii];
+    if (id < 0 || id >= p.num_blocks) {  // never dereference outside the pool
+      id = 0;
+      bad |= 1u << st;
+    } else {
+      bad &= ~(1u << st);
+    }
+    const int64_t off = (int64_t)id * blk_bytes + (int64_t)LY::kTileBytes * inf->kvh;
+    const char* kt = kc + off;
+    const char* vt = vc + off;
+    const uint32_t ks = ring + st * LY::kStageBytes;
+    const uint32_t vs = ks + LY::kTileBytes;
+#pragma unroll
+    for (int c = 0; c < kCopies; ++c) {
+      const int idx = lane + 32 * c;
+      const int row = idx / kChunks, ch = idx % kChunks;
+      cp_async16(ks + (row * kChunks + (ch ^ k_swz(row))) * 16, kt + idx * 16);
+      cp_async16(vs + (row * kChunks + (ch ^ v_swz(row))) * 16, vt + idx * 16);
+    }
+    cp_async_commit();
+    if (lane == 0) {
+      my_meta[2 * st] = ip;
+      my_meta[2 * st + 1] = ii;
+    }
+    ++n_issued;
+    ii += kWarps;
+    return true;
+  };
+
+  // per-piece state of this warp
+  int cur = -1;  // piece being accumulated
+  uint32_t qa[NC][2], qb[NC][2];
+  float o[NT][4];
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+  int lim_a = 0, lim_b = 0, first_masked = 0;
+
+  // The warp's part of piece pc is done: its (max, sum, O) go to the merge
+  // slot; the last warp to arrive merges and stores the piece's result.
+  auto flush = [&](int pc, const PieceInfo* inf) -> bool {
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    if (kRows16) {
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    }
+    // the merge slot holds one piece at a time: the previous one must be merged
+    if (!spin_until([&] { return *(volatile int*)&ctl.merged >= pc - 1; }, vabort, status))
+      return false;
+    if (q4 == 0) {
+      if (r < kMaxRows) { msl_m[warp * kMaxRows + r] = m_a; msl_l[warp * kMaxRows + r] = l_a; }
+      if (kRows16 && r + 8 < kMaxRows) {
+        msl_m[warp * kMaxRows + r + 8] = m_b;
+        msl_l[warp * kMaxRows + r + 8] = l_b;
+      }
+    }
+    float* mo = msl_o + warp * kMaxRows * D;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int d = out_dim(nt, 2 * q4 + c);
+        if (r < kMaxRows) mo[r * D + d] = o[nt][c];
+        if (kRows16 && r + 8 < kMaxRows) mo[(r + 8) * D + d] = o[nt][2 + c];
+      }
+    }
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      const int arrived = atomicAdd(&ctl.count, 1) + 1;
+      last = arrived == min(kWarps, inf->nb);
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return true;
+    __threadfence_block();  // every lane sees the other warps' parts
+
+    // ---- merge the warps' parts of the piece
+    const int nw = min(kWarps, inf->nb);
+    const int rows = inf->rows;
+    const int s = inf->s, kvh = inf->kvh, rg = inf->rg;
+    const int unit = s * p.num_kv_heads + kvh;
+    __nv_bfloat16* out = (__nv_bfloat16*)p.out;
+    constexpr int D4 = D / 4;
+    const bool direct = inf->nparts == 1;
+    const int64_t slot0 = ((int64_t)unit * p.max_parts + inf->j * p.row_groups + rg) * kDecodeRows;
+    for (int e = lane; e < rows * D4; e += 32) {
+      const int i = e / D4, d4 = e % D4;
+      float M = -INFINITY;
+      for (int w = 0; w < nw; ++w) M = fmaxf(M, msl_m[w * kMaxRows + i]);
+      const float base = (M == -INFINITY) ? 0.f : M;
+      float Ls = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int w = 0; w < nw; ++w) {
+        const float f = exp2f(msl_m[w * kMaxRows + i] - base);
+        Ls += msl_l[w * kMaxRows + i] * f;
+        const float4 v = *reinterpret_cast<const float4*>(msl_o + (w * kMaxRows + i) * D + 4 * d4);
+        acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+      }
+      if (direct) {
+        const int gi = inf->row0 + i;
+        const int64_t tok = inf->q0 + gi / G, head = (int64_t)kvh * G + gi % G;
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        uint2 pk;
+        pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
+      } else {
+        reinterpret_cast<float4*>(p.ws_o)[(slot0 + i) * D4 + d4] = acc;
+        if (d4 == 0) reinterpret_cast<float2*>(p.ws_ml)[slot0 + i] = make_float2(M, Ls);
+      }
+    }
+    if (!direct) {
+      // ---- the last arriving piece of the unit merges all of its partials
+      __threadfence();
+      __syncwarp();
+      int ulast = 0;
+      int* counter = p.ws_counter + unit * kDecodeRowGroups + rg;
+      if (lane == 0) ulast = atomicAdd(counter, 1) == inf->nparts - 1;
+      ulast = __shfl_sync(0xffffffffu, ulast, 0);
+      if (ulast) {
+        __threadfence();  // every lane sees the other pieces' partials
+        const int np = inf->nparts;
+        const int64_t uslot = ((int64_t)unit * p.max_parts + rg) * kDecodeRows;
+        const int64_t step = (int64_t)p.row_groups * kDecodeRows;  // next part, same row
+        const float2* pml = reinterpret_cast<const float2*>(p.ws_ml);
+        // per row: merged max and 1 / merged sum, kept in the (now read) merge slot
+        float* rM = msl_m;
+        float* rI = msl_l;
+        for (int i = 0; i < rows; ++i) {
+          float M = -INFINITY;
+          for (int q = lane; q < np; q += 32) M = fmaxf(M, __ldcg(pml + uslot + q * step + i).x);
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+          const float base = (M == -INFINITY) ? 0.f : M;
+          float Ls = 0.f;
+          for (int q = lane; q < np; q += 32) {
+            const float2 ml = __ldcg(pml + uslot + q * step + i);
+            Ls += ml.y * exp2f(ml.x - base);
+          }
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o2);
+          if (lane == 0) {
+            rM[i] = base;
+            rI[i] = Ls > 0.f ? 1.f / Ls : 0.f;
+          }
+        }
+        __syncwarp();
+        const float4* po = reinterpret_cast<const float4*>(p.ws_o);
+        for (int e = lane; e < rows * D4; e += 32) {
+          const int i = e / D4, d4 = e % D4;
+          const float base = rM[i];
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+          for (int q = 0; q < np; ++q) {
+            const int64_t sl = uslot + q * step + i;
+            const float f = exp2f(__ldcg(pml + sl).x - base);
+            const float4 v = __ldcg(po + sl * D4 + d4);
+            acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+          }
+          const float inv = rI[i];
+          const int gi = inf->row0 + i;
+          const int64_t tok = inf->q0 + gi / G, head = (int64_t)kvh * G + gi % G;
+          uint2 pk;
+          pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+          pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+          *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
+        }
+        if (lane == 0) *counter = 0;  // ready for the next call
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      ctl.count = 0;
+      __threadfence_block();
+      *(volatile int*)&ctl.merged = pc;
+    }
+    __syncwarp();
+    return true;
+  };
+
+  while (true) {
+    // keep kStages blocks in flight; wait for a piece to be published only
+    // when nothing is in flight
+    while (!issue_done && n_issued - n_comp < kStages) {
+      if (!try_issue(n_issued == n_comp)) break;
+    }
+    if (n_issued == n_comp) break;  // the list is exhausted (or the CTA aborted)
+    cp_async_wait_pending<kStages>(n_issued - n_comp - 1);
+    __syncwarp();  // every lane's copies of the oldest stage have landed
+
+    const int st = n_comp % kStages;
+    const int pc = my_meta[2 * st], i = my_meta[2 * st + 1];
+    const PieceInfo* inf = slot_info(pc);
+    const int L = inf->L;
+    if (pc != cur) {
+      // ---- a new piece: its query rows as the A operand (rows r and r+8), D
+      // axis permuted as the K chunks; fresh running max, sum and O
+      cur = pc;
+      const uint32_t qs = slot_q(pc);
+#pragma unroll
+      for (int jp = 0; jp < NJ; ++jp) {
+        uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
+        if (r < kMaxRows) xa = lds128(qs + (r * kChunks + 4 * jp + q4) * 16);
+        if (kRows16 && r + 8 < kMaxRows) xb = lds128(qs + ((r + 8) * kChunks + 4 * jp + q4) * 16);
+        qa[2 * jp][0] = xa.x; qa[2 * jp][1] = xa.y; qa[2 * jp + 1][0] = xa.z; qa[2 * jp + 1][1] = xa.w;
+        qb[2 * jp][0] = xb.x; qb[2 * jp][1] = xb.y; qb[2 * jp + 1][0] = xb.z; qb[2 * jp + 1][1] = xb.w;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+      m_a = m_b = -INFINITY;
+      l_a = l_b = 0.f;
+      const int rows = inf->rows, ql = inf->ql;
+      // causal limit of rows r and r+8: query j sees keys <= L - ql + j
+      lim_a = L - ql + (inf->row0 + min(r, rows - 1)) / G;
+      lim_b = L - ql + (inf->row0 + min(r + 8, rows - 1)) / G;
+      first_masked = L - ql + 1;  // keys at or beyond this may be masked for some row
+    }
+
+    const int blk = inf->blk_begin + i;
+    const bool blk_ok = !((bad >> st) & 1u);
+    const uint32_t ks = ring + st * LY::kStageBytes;
+    const uint32_t vs = ks + LY::kTileBytes;
+
+    // ---- S = Q K^T (two 8-key halves of the block)
+    float sc[2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      sc[h][0] = sc[h][1] = sc[h][2] = sc[h][3] = 0.f;
+      const int row = 8 * h + r;
+#pragma unroll
+      for (int jp = 0; jp < NJ; ++jp) {
+        const uint4 kx = lds128(ks + (row * kChunks + ((4 * jp + q4) ^ k_swz(row))) * 16);
+        mma_16816(sc[h], qa[2 * jp][0], kRows16 ? qb[2 * jp][0] : 0u, qa[2 * jp][1],
+                  kRows16 ? qb[2 * jp][1] : 0u, kx.x, kx.y);
+        mma_16816(sc[h], qa[2 * jp + 1][0], kRows16 ? qb[2 * jp + 1][0] : 0u,
+                  qa[2 * jp + 1][1], kRows16 ? qb[2 * jp + 1][1] : 0u, kx.z, kx.w);
+      }
+    }
+    // ---- V words: keys 2q4, 2q4+1, 2q4+8, 2q4+9; 8 dims 64u+8r.. each
+    uint4 vw[4][NV];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = 2 * q4 + (e & 1) + 8 * (e >> 1);
+#pragma unroll
+      for (int u = 0; u < NV; ++u)
+        vw[e][u] = lds128(vs + (tok * kChunks + ((8 * u + r) ^ v_swz(tok))) * 16);
+    }
+    // slots of the last block past seq_len (and blocks outside the pool) may
+    // hold anything, NaN included: their V words become zeros so that the
+    // zero weights below cannot turn them into NaN in the P.V product
+    if (blk * kBlockSize + kBlockSize > L || !blk_ok) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = blk * kBlockSize + 2 * q4 + (e & 1) + 8 * (e >> 1);
+        if (!blk_ok || key >= L) {
+#pragma unroll
+          for (int u = 0; u < NV; ++u) vw[e][u] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+    // ---- scale, mask, online softmax
+    const int key0 = blk * kBlockSize + 2 * q4;  // keys key0, +1 (half 0), key0+8, +9 (half 1)
+    const bool tail = (blk * kBlockSize + kBlockSize > first_masked) || !blk_ok;
+    float xa[4], xb[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = key0 + (e & 1) + 8 * (e >> 1);
+      xa[e] = sc[e >> 1][e & 1] * p.scale_log2;
+      xb[e] = sc[e >> 1][2 + (e & 1)] * p.scale_log2;
+      if (tail) {
+        if (!blk_ok || key > lim_a) xa[e] = -INFINITY;
+        if (!blk_ok || key > lim_b) xb[e] = -INFINITY;
+      }
+    }
+    float bm_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
+    bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 1));
+    bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 2));
+    const float mn_a = fmaxf(m_a, bm_a);
+    const float base_a = (mn_a == -INFINITY) ? 0.f : mn_a;
+    const float al_a = exp2f(m_a - base_a);
+    float pa[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pa[e] = exp2f(xa[e] - base_a);
+    l_a = l_a * al_a + (pa[0] + pa[1]) + (pa[2] + pa[3]);
+    m_a = mn_a;
+    float pb[4] = {0.f, 0.f, 0.f, 0.f};
+    float al_b = 1.f;
+    if (kRows16) {
+      float bm_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
+      bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 1));
+      bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 2));
+      const float mn_b = fmaxf(m_b, bm_b);
+      const float base_b = (mn_b == -INFINITY) ? 0.f : mn_b;
+      al_b = exp2f(m_b - base_b);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pb[e] = exp2f(xb[e] - base_b);
+      l_b = l_b * al_b + (pb[0] + pb[1]) + (pb[2] + pb[3]);
+      m_b = mn_b;
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      o[nt][0] *= al_a; o[nt][1] *= al_a;
+      if (kRows16) { o[nt][2] *= al_b; o[nt][3] *= al_b; }
+    }
+    // ---- O += P V
+    const uint32_t pa0 = pack_bf16x2(pa[0], pa[1]), pa2 = pack_bf16x2(pa[2], pa[3]);
+    const uint32_t pb1 = kRows16 ? pack_bf16x2(pb[0], pb[1]) : 0u;
+    const uint32_t pb3 = kRows16 ? pack_bf16x2(pb[2], pb[3]) : 0u;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int u = nt / 8, idx = nt % 8;
+      const uint32_t sel = (idx & 1) ? 0x7632u : 0x5410u;
+      const uint32_t b0 = __byte_perm(word(vw[0][u], idx >> 1), word(vw[1][u], idx >> 1), sel);
+      const uint32_t b1 = __byte_perm(word(vw[2][u], idx >> 1), word(vw[3][u], idx >> 1), sel);
+      mma_16816(o[nt], pa0, pb1, pa2, pb3, b0, b1);
+    }
+    ++n_comp;
+    __syncwarp();  // every lane is done with this stage before it is refilled
+    if (i + kWarps >= inf->nb) {  // this warp's last block of the piece
+      if (!flush(pc, inf)) break;
+    }
+  }
+  cp_async_wait<0>();  // no copy may still target the ring when the CTA exits
+}
+
+template <int D, int kMaxRows, bool kWriteCache>
+cudaError_t launch_one(const AttnParams& p, const DecodeWork& work, int grid,
+                       cudaStream_t stream) {
+  using LY = DecodeLayout<D, kMaxRows>;
+  auto kernel = decode_persistent_kernel<D, kMaxRows, kWriteCache>;
+  static std::atomic<int> smem_done[64];
+  cudaError_t e = raise_smem_limit(kernel, LY::total, smem_done);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3((LY::kWarps + 1) * 32);
+  cfg.dynamicSmemBytes = LY::total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p, work);
+}
+
+template <int D, bool kWriteCache>
+cudaError_t launch_rows(const AttnParams& p, const DecodeWork& work, int grid, int max_rows,
+                        cudaStream_t stream) {
+  if (max_rows <= 4) return launch_one<D, 4, kWriteCache>(p, work, grid, stream);
+  if (max_rows <= 8) return launch_one<D, 8, kWriteCache>(p, work, grid, stream);
+  return launch_one<D, 16, kWriteCache>(p, work, grid, stream);
+}
+
+// ------------------------------------------------------------------ piece lists
+
+// Decode-class test and block count of sequence s (0: no decode work).
+__host__ __device__ __forceinline__ int decode_blocks(int ql, int L, int group, int max_seq_len,
+                                                      int max_blocks_per_seq) {
+  if (ql <= 0 || ql > L || ql * group > kDecodeMaxRows || L > max_seq_len) return 0;
+  const int nblk = (L + kBlockSize - 1) / kBlockSize;
+  return nblk <= max_blocks_per_seq ? nblk : 0;
+}
+
+// Blocks per piece: about total / (kDecodePiecesPerCta * ctas), so that every
+// CTA gets a few pieces, and no more than kDecodeMaxPieceBytes of K+V, so
+// that the last pieces of a big step stay short; but never fewer than the
+// workspace's partial slots allow for the longest unit.
+__host__ __device__ __forceinline__ int choose_piece_blocks(long long total_blocks, int max_nblk,
+                                                            int ctas, int slots_per_unit,
+                                                            int head_dim) {
+  long long want = (total_blocks + (long long)kDecodePiecesPerCta * ctas - 1) /
+                   ((long long)kDecodePiecesPerCta * ctas);
+  if (want < kDecodeMinPieceBlocks) want = kDecodeMinPieceBlocks;
+  const long long cap = kDecodeMaxPieceBytes / (2 * kBlockSize * head_dim * 2);
+  if (want > cap) want = cap;
+  const long long need = (max_nblk + slots_per_unit - 1) / max(1, slots_per_unit);
+  if (want < need) want = need;
+  if (want > kDecodeMaxPieceBlocks) want = kDecodeMaxPieceBlocks;
+  return (int)want;
+}
+
+__host__ __device__ __forceinline__ int4 make_piece(int s, int kvh, int rg, int j, int ql, int L,
+                                                    int q0) {
+  return make_int4(s, (ql << 24) | (rg << 22) | (kvh << 12) | j, L, q0);
+}
+
+// One CTA: the piece list of every decode-class sequence, written to the
+// workspace (count, blocks per piece, then the pieces, largest first).
+__global__ void __launch_bounds__(1024)
+decode_plan_kernel(const AttnParams p, int ctas, int head_dim) {
+  __shared__ unsigned long long sh_total;
+  __shared__ int sh_max_nblk, sh_P, sh_full, sh_count;
+  __shared__ int hist[kDecodeMaxPieceBlocks + 1];  // tail pieces by size, then offsets
+  // the decode kernel may be launched at once: it waits for this grid before
+  // it reads the list
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x == 0) {
+    sh_total = 0;
+    sh_max_nblk = 0;
+    sh_full = 0;
+  }
+  for (int i = threadIdx.x; i <= kDecodeMaxPieceBlocks; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int G = p.group, H = p.num_kv_heads;
+  auto groups_of = [&](int ql) { return (ql * G + kDecodeRows - 1) / kDecodeRows; };
+  // pass 1: total blocks over the units, longest unit
+  unsigned long long tot = 0;
+  int mx = 0;
+  for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
+    const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
+    const int nblk = decode_blocks(ql, L, G, p.max_seq_len, p.max_blocks_per_seq);
+    if (!nblk || ql * G > p.decode_rows) continue;
+    tot += (unsigned long long)nblk * H * groups_of(ql);
+    mx = max(mx, nblk);
+  }
+  atomicAdd(&sh_total, tot);
+  atomicMax(&sh_max_nblk, mx);
+  __syncthreads();
+  if (threadIdx.x == 0)
+    sh_P = choose_piece_blocks((long long)sh_total, sh_max_nblk, ctas,
+                               p.max_parts / max(1, p.row_groups), head_dim);
+  __syncthreads();
+  const int P = sh_P;
+  // pass 2: count the full pieces and the tail pieces by size
+  int full = 0;
+  for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
+    const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
+    const int nblk = decode_blocks(ql, L, G, p.max_seq_len, p.max_blocks_per_seq);
+    if (!nblk || ql * G > p.decode_rows) continue;
+    const int units = H * groups_of(ql);
+    full += units * (nblk / P);
+    if (nblk % P) atomicAdd(&hist[nblk % P], units);
+  }
+  atomicAdd(&sh_full, full);
+  __syncthreads();
+  if (threadIdx.x == 0) {  // offsets: full pieces from 0, then tails by falling size
+    int run = sh_full;
+    for (int sz = P - 1; sz >= 1; --sz) {
+      const int c = hist[sz];
+      hist[sz] = run;
+      run += c;
+    }
+    sh_count = min(run, p.max_pieces);
+    sh_full = 0;  // becomes the running offset of the full pieces
+    p.ws_header[kWsPieceCount] = sh_count;
+    p.ws_header[kWsPieceBlocks] = P;
+  }
+  __syncthreads();
+  // pass 3: scatter
+  for (int s = threadIdx.x; s < p.num_seqs; s += blockDim.x) {
+    const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
+    const int nblk = decode_blocks(ql, L, G, p.max_seq_len, p.max_blocks_per_seq);
+    if (!nblk || ql * G > p.decode_rows) continue;
+    const int ng = groups_of(ql), nf = nblk / P;
+    if (nf) {
+      int at = atomicAdd(&sh_full, H * ng * nf);
+      for (int kvh = 0; kvh < H; ++kvh)
+        for (int rg = 0; rg < ng; ++rg)
+          for (int j = 0; j < nf; ++j, ++at)
+            if (at < p.max_pieces) p.ws_pieces[at] = make_piece(s, kvh, rg, j, ql, L, q0);
+    }
+    if (nblk % P) {
+      int at = atomicAdd(&hist[nblk % P], H * ng);
+      for (int kvh = 0; kvh < H; ++kvh)
+        for (int rg = 0; rg < ng; ++rg, ++at)
+          if (at < p.max_pieces) p.ws_pieces[at] = make_piece(s, kvh, rg, nf, ql, L, q0);
+    }
+  }
+}
+
+// The same list built on the host from its copies of the lengths; false when
+// it holds more pieces than a kernel parameter carries.
+bool host_piece_list(DecodeWork* work, const AttnParams& p, const int32_t* seq_lens_host,
+                     const int32_t* query_start_loc_host, int ctas, int head_dim) {
+  const int G = p.group, H = p.num_kv_heads;
+  auto groups_of = [&](int ql) { return (ql * G + kDecodeRows - 1) / kDecodeRows; };
+  long long total = 0;
+  int mx = 0;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int ql = query_start_loc_host[s + 1] - query_start_loc_host[s];
+    const int nblk = decode_blocks(ql, seq_lens_host[s], G, p.max_seq_len, p.max_blocks_per_seq);
+    if (!nblk || ql * G > p.decode_rows) continue;
+    total += (long long)nblk * H * groups_of(ql);
+    mx = max(mx, nblk);
+  }
+  const int P =
+      choose_piece_blocks(total, mx, ctas, p.max_parts / max(1, p.row_groups), head_dim);
+  static thread_local int hist[kDecodeMaxPieceBlocks + 1];
+  for (int i = 0; i <= P; ++i) hist[i] = 0;
+  long long full = 0;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int ql = query_start_loc_host[s + 1] - query_start_loc_host[s];
+    const int nblk = decode_blocks(ql, seq_lens_host[s], G, p.max_seq_len, p.max_blocks_per_seq);
+    if (!nblk || ql * G > p.decode_rows) continue;
+    const int units = H * groups_of(ql);
+    full += (long long)units * (nblk / P);
+    if (nblk % P) hist[nblk % P] += units;
+  }
+  long long run = full;
+  for (int sz = P - 1; sz >= 1; --sz) {
+    const int c = hist[sz];
+    hist[sz] = (int)min(run, (long long)INT32_MAX);
+    run += c;
+  }
+  if (run > kDecodeParamPieces) return false;
+  int at_full = 0;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int q0 = query_start_loc_host[s], ql = query_start_loc_host[s + 1] - q0;
+    const int L = seq_lens_host[s];
+    const int nblk = decode_blocks(ql, L, G, p.max_seq_len, p.max_blocks_per_seq);
+    if (!nblk || ql * G > p.decode_rows) continue;
+    const int ng = groups_of(ql), nf = nblk / P;
+    for (int kvh = 0; kvh < H; ++kvh)
+      for (int rg = 0; rg < ng; ++rg) {
+        for (int j = 0; j < nf; ++j) work->items[at_full++] = make_piece(s, kvh, rg, j, ql, L, q0);
+        if (nblk % P) work->items[hist[nblk % P]++] = make_piece(s, kvh, rg, nf, ql, L, q0);
+      }
+  }
+  work->count = (int)run;
+  work->piece_blocks = P;
+  work->from_ws = 0;
+  return true;
+}
+
+template <int D, int kMaxRows>
+int max_ctas_one() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  using LY = DecodeLayout<D, kMaxRows>;
+  auto kernel = decode_persistent_kernel<D, kMaxRows, false>;
+  static std::atomic<int> smem_done[64];
+  int per_sm = 0;
+  if (raise_smem_limit(kernel, LY::total, smem_done) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, (LY::kWarps + 1) * 32,
+                                                    LY::total) != cudaSuccess ||
+      per_sm <= 0)
+    per_sm = 1;
+  n = per_sm * device_sm_count();
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+int max_ctas(int head_dim, int max_rows) {
+  if (head_dim == 64)
+    return max_rows <= 4 ? max_ctas_one<64, 4>() : max_rows <= 8 ? max_ctas_one<64, 8>()
+                                                                 : max_ctas_one<64, 16>();
+  return max_rows <= 4 ? max_ctas_one<128, 4>() : max_rows <= 8 ? max_ctas_one<128, 8>()
+                                                                : max_ctas_one<128, 16>();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_lens_host,
+                          const int32_t* query_start_loc_host, cudaStream_t stream,
+                          int max_ctas_allowed) {
+  if (p.num_seqs == 0) return cudaSuccess;
+  const int max_rows = max(1, min(p.decode_rows, kDecodeRows));  // rows of one unit at most
+  const int ctas = max(1, min(max_ctas(head_dim, max_rows), max_ctas_allowed));
+  static thread_local DecodeWork work;  // 16 KB: kept off the stack
+  int grid = ctas;
+  if (seq_lens_host && query_start_loc_host &&
+      host_piece_list(&work, p, seq_lens_host, query_start_loc_host, ctas, head_dim)) {
+    if (work.count == 0) return cudaSuccess;
+    grid = min(ctas, work.count);
+  } else {
+    work.count = 0;
+    work.piece_blocks = 0;
+    work.from_ws = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(1024);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_plan_kernel, p, ctas, head_dim);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e;
+  const bool wc = p.slot_mapping != nullptr;
+  if (head_dim == 64)
+    e = wc ? launch_rows<64, true>(p, work, grid, max_rows, stream)
+           : launch_rows<64, false>(p, work, grid, max_rows, stream);
+  else
+    e = wc ? launch_rows<128, true>(p, work, grid, max_rows, stream)
+           : launch_rows<128, false>(p, work, grid, max_rows, stream);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace pa

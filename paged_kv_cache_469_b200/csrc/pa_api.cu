@@ -9,38 +9,13 @@ namespace pa {
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Split-K partitions.  The workspace is laid out for partitions as short as
-// part_tokens_floor(max_seq_len) keys: a power of two in [PA_PART_MIN,
-// PA_PART_MAX], at least a quarter of max_seq_len, so that a sequence never
-// needs more than four partitions unless it is longer than 4 * PA_PART_MAX.
-// Each call then picks its own partition length, no shorter than that floor
-// and no longer than PA_PART_MAX: about the step's total keys divided by the
-// number of decode CTAs the GPU holds at once (one full wave; the hardware
-// hands later partitions to SMs as they free up), so that a small step still
-// keeps every SM streaming and no partition is much longer than the rest.
-#ifndef PA_PART_MIN
-#define PA_PART_MIN 512
-#endif
-#ifndef PA_PART_MAX
-#define PA_PART_MAX 2048
-#endif
-static int part_tokens_floor(int max_seq_len) {
-  int part = PA_PART_MIN;
-  while (part < PA_PART_MAX && (long)part * 4 < (long)max_seq_len) part *= 2;
-  return part;
-}
-#ifndef PA_DECODE_WAVES
-#define PA_DECODE_WAVES 0.5
-#endif
-static int part_tokens_for_step(long total_unit_keys, int wave_ctas, int floor_tokens) {
-  const long ctas = (long)(PA_DECODE_WAVES * (wave_ctas > 0 ? wave_ctas : 1)) + 1;
-  long part = (total_unit_keys + ctas - 1) / ctas;
-  part = (part + kBlockSize - 1) / kBlockSize * kBlockSize;
-  if (part < floor_tokens) part = floor_tokens;
-  if (part > PA_PART_MAX) part = PA_PART_MAX;
-  return (int)part;
-}
-
+// Split-K partial slots.  A decode unit (sequence, kv-head, row group) of
+// nblk blocks is cut into pieces of P blocks, P chosen per launch; each piece
+// of a unit that has more than one keeps an fp32 partial in the workspace.
+// The workspace holds max_parts slots per (sequence, kv-head), shared by its
+// row groups: kDecodePartsBase plus one per kDecodePartsPerBlocks blocks of
+// the longest sequence, so that short sequences can be cut finely and long
+// ones into pieces of a few hundred blocks at most.
 int device_sm_count() {
   static std::atomic<int> n[64];
   int dev = 0;
@@ -57,22 +32,25 @@ int device_sm_count() {
 WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_seq_len) {
   WorkspaceLayout w{};
-  w.part_tokens = part_tokens_floor(max_seq_len);
-  // a slot per (partition, row group): at least one partition for each of the
-  // row groups a multi-token decode may need
-  w.max_parts = max(kDecodeRowGroups, (max_seq_len + w.part_tokens - 1) / w.part_tokens);
+  const long max_blocks = ((long)max_seq_len + kBlockSize - 1) / kBlockSize;
+  w.max_parts = (int)min((long)INT32_MAX,
+                         kDecodePartsBase +
+                             (max_blocks + kDecodePartsPerBlocks - 1) / kDecodePartsPerBlocks);
   // prefill items: at most ceil(q_len / 128) <= ceil(max_seq_len / 128) per sequence and q-head
   const long items = (long)num_seqs * ((max_seq_len + kPrefillQTile - 1) / kPrefillQTile) *
                      num_q_heads;
   w.max_items = (int)min(items, (long)(1 << 30));
   const size_t units = (size_t)num_seqs * num_kv_heads;
+  // the device-built piece list: at most one piece per partial slot
+  w.max_pieces = (int)min(units * (size_t)w.max_parts, (size_t)(1 << 30));
   const size_t slots = units * w.max_parts * kDecodeRows;
   w.status_off = 0;
   w.counter_off = 256;
   // one arrival counter per (sequence, kv-head, row group)
   w.o_off = align_up(w.counter_off + units * kDecodeRowGroups * sizeof(int), 256);
   w.ml_off = align_up(w.o_off + slots * head_dim * sizeof(float), 256);
-  w.items_off = align_up(w.ml_off + slots * 2 * sizeof(float), 256);
+  w.pieces_off = align_up(w.ml_off + slots * 2 * sizeof(float), 256);
+  w.items_off = align_up(w.pieces_off + (size_t)w.max_pieces * 16, 256);
   w.total = align_up(w.items_off + (size_t)(w.max_items + 1) * 16, 256);
   return w;
 }
@@ -115,6 +93,17 @@ extern "C" int pa_reshape_and_cache(const void* k, const void* v, void* k_cache,
 
 static bool aligned_to(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
+// A byte range [p, p + n) of caller memory (n = 0: empty, overlaps nothing).
+struct Range {
+  const void* p;
+  size_t n;
+  bool overlaps(const Range& o) const {
+    if (!p || !o.p || n == 0 || o.n == 0) return false;
+    const uintptr_t a = (uintptr_t)p, b = (uintptr_t)o.p;
+    return a < b + o.n && b < a + n;
+  }
+};
+
 extern "C" int pa_plan_step(const int32_t* free_queue, int queue_len, int32_t* planner_state,
                             const int32_t* num_computed, const int32_t* query_lens,
                             int num_seqs, int32_t* block_tables, int max_blocks_per_seq,
@@ -132,6 +121,17 @@ extern "C" int pa_plan_step(const int32_t* free_queue, int queue_len, int32_t* p
       !aligned_to(block_tables, 4) || !aligned_to(seq_lens, 4) || !aligned_to(free_queue, 4) ||
       !aligned_to(slot_mapping, 8))
     return PA_ERR_INVALID;
+  // The kernel's CTAs read num_computed and query_lens in full while other
+  // CTAs already write seq_lens, query_start_loc and the slots: an output that
+  // shares memory with an input would be read half old, half new.
+  if (num_seqs > 0) {
+    const Range in_nc{num_computed, (size_t)num_seqs * 4}, in_ql{query_lens, (size_t)num_seqs * 4};
+    const Range outs[3] = {{seq_lens, (size_t)num_seqs * 4},
+                           {query_start_loc, ((size_t)num_seqs + 1) * 4},
+                           {slot_mapping, (size_t)max_tokens * 8}};
+    for (const Range& o : outs)
+      if (o.overlaps(in_nc) || o.overlaps(in_ql)) return PA_ERR_INVALID;
+  }
   cudaError_t e = launch_plan_step(free_queue, queue_len, planner_state, num_computed,
                                    query_lens, num_seqs, block_tables, max_blocks_per_seq,
                                    seq_lens, query_start_loc, slot_mapping, max_tokens,
@@ -167,12 +167,50 @@ extern "C" int pa_workspace_init(void* workspace, size_t workspace_bytes,
 
 namespace {
 
+// Rates one SM sustains on its own, used only to split the SMs between the
+// two classes of a mixed step: the tensor-core prefill kernel (bf16 flops of
+// unmasked query-key pairs per second) and the decode kernel (K/V bytes per
+// second when every SM streams).
+constexpr double kPrefillFlopsPerSm = 5.0e12;
+constexpr double kDecodeBytesPerSm = 46.0e9;
+
+// A side stream and two events, per thread and device, for the calls that run
+// the prefill kernel beside the decode kernel.  Created on the first such call
+// outside a stream capture; a capture that would need to create them runs the
+// kernels one after the other instead.
+struct ForkStreams {
+  cudaStream_t side = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+};
+
+ForkStreams* fork_streams(cudaStream_t st) {
+  static thread_local ForkStreams per_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  ForkStreams& f = per_dev[dev];
+  if (f.side && f.start && f.done) return &f;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+    return nullptr;
+  if ((!f.side && cudaStreamCreateWithFlags(&f.side, cudaStreamNonBlocking) != cudaSuccess) ||
+      (!f.start && cudaEventCreateWithFlags(&f.start, cudaEventDisableTiming) != cudaSuccess) ||
+      (!f.done && cudaEventCreateWithFlags(&f.done, cudaEventDisableTiming) != cudaSuccess))
+    return nullptr;
+  return &f;
+}
+
 // The new tokens' K/V rows a call writes into the cache before it reads it
 // (pa_attention_varlen_write_cache); all null for pa_attention_varlen.
 struct CacheWrite {
   const void* k_new = nullptr;
   const void* v_new = nullptr;
   const int64_t* slot_mapping = nullptr;
+};
+
+struct CallOptions {
+  // may run the two classes of a mixed step side by side on a side stream
+  // (created on first use); false for callers that must not create anything
+  bool allow_fork = true;
 };
 
 int attention_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -182,7 +220,7 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
                    int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
                    void* workspace, size_t workspace_bytes, const int32_t* seq_lens_host,
                    const int32_t* query_start_loc_host, struct CUstream_st* stream,
-                   const CacheWrite& cw) {
+                   const CacheWrite& cw, const CallOptions& opt) {
   const bool write_cache = cw.slot_mapping != nullptr;
   // ---- scalar checks
   if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || max_seq_len < 0 ||
@@ -208,6 +246,7 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
   bool any_decode = true, any_prefill = true;
   int prefill_items = -1;  // unknown without the host copies
   long decode_keys = -1;   // sum of the decode-class sequences' lengths, when known
+  double prefill_flops = 0;  // of the prefill-class sequences, when known
   int decode_rows = min(max_query_len * group, kDecodeMaxRows);  // most rows of one of them
   if (seq_lens_host && query_start_loc_host) {
     if (query_start_loc_host[0] != 0 || query_start_loc_host[num_seqs] != num_tokens)
@@ -228,6 +267,9 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
       } else {
         any_prefill = true;
         prefill_items += (ql + kPrefillQTile - 1) / kPrefillQTile * num_q_heads;
+        // unmasked (query, key) pairs: ql * (L - ql) of cached context + ql (ql + 1) / 2
+        prefill_flops += 4.0 * head_dim * num_q_heads *
+                         ((double)ql * (L - ql) + (double)ql * (ql + 1) / 2);
       }
     }
   } else if (max_query_len * group <= kDecodeMaxRows) {
@@ -237,9 +279,6 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
   const WorkspaceLayout w =
       workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len);
   if (w.max_parts > kDecodeMaxParts) return PA_ERR_UNSUPPORTED;
-  // the decode grid holds one sequence per z index
-  if (any_decode && dtype == PA_DTYPE_BF16 && num_seqs > kDecodeMaxSeqs)
-    return PA_ERR_UNSUPPORTED;
   AttnParams p{};
   p.out = out;
   p.q = q;
@@ -250,19 +289,19 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
   p.query_start_loc = query_start_loc;
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.max_seq_len = max_seq_len;
-  p.max_parts = w.max_parts;  // the workspace's partitions per (sequence, kv-head)
+  p.max_parts = w.max_parts;  // the workspace's partial slots per (sequence, kv-head)
+  p.max_pieces = w.max_pieces;
+  p.row_groups = max(1, (decode_rows + kDecodeRows - 1) / kDecodeRows);
+  p.decode_rows = decode_rows;
+  // the longest sequence must fit the slots of its (sequence, kv-head) in
+  // pieces of at most kDecodeMaxPieceBlocks blocks
   {
-    p.row_groups = max(1, (decode_rows + kDecodeRows - 1) / kDecodeRows);
-    p.decode_rows = decode_rows;
-    const int rows = max(1, min(decode_rows, kDecodeRows));  // per CTA
-    const long keys = decode_keys >= 0 ? decode_keys : (long)num_seqs * (max_seq_len / 2 + 1);
-    int part = part_tokens_for_step(keys * num_kv_heads * p.row_groups,
-                                    decode_wave_ctas(head_dim, rows), w.part_tokens);
-    // the slots of one (sequence, kv-head) hold every (partition, row group)
-    const int parts_cap = max(1, w.max_parts / p.row_groups);
-    const long need = ((long)max_seq_len + parts_cap - 1) / parts_cap;
-    if (need > part) part = (int)((need + kBlockSize - 1) / kBlockSize * kBlockSize);
-    p.part_tokens = part;
+    const long max_blocks = ((long)max_seq_len + kBlockSize - 1) / kBlockSize;
+    const long slots_per_unit = w.max_parts / p.row_groups;
+    if (any_decode && dtype == PA_DTYPE_BF16 &&
+        (slots_per_unit < 1 ||
+         (max_blocks + slots_per_unit - 1) / slots_per_unit > kDecodeMaxPieceBlocks))
+      return PA_ERR_UNSUPPORTED;
   }
   p.num_seqs = num_seqs;
   p.num_tokens = num_tokens;
@@ -298,9 +337,11 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
 
   char* ws = (char*)workspace;
   p.ws_status = (int*)(ws + w.status_off);
+  p.ws_header = p.ws_status;
   p.ws_counter = (int*)(ws + w.counter_off);
   p.ws_o = (float*)(ws + w.o_off);
   p.ws_ml = (float*)(ws + w.ml_off);
+  p.ws_pieces = (int4*)(ws + w.pieces_off);
   p.ws_items = (int4*)(ws + w.items_off);
   p.max_items = w.max_items;
   if (fused_write) {
@@ -308,13 +349,46 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
     p.v_new = cw.v_new;
     p.slot_mapping = cw.slot_mapping;
   }
+  const int sms = device_sm_count();
+  // A step with both classes of work (known from the host copies) runs them
+  // side by side: the prefill kernel on a side stream, on a share of the SMs
+  // proportional to its share of the step's work, the decode kernel on the
+  // rest, joined back into `stream` before the call returns.
+  ForkStreams* fork = nullptr;
+  int prefill_ctas = sms, decode_ctas = sms;
+  if (opt.allow_fork && any_decode && any_prefill && prefill_flops > 0 && decode_keys > 0) {
+    fork = fork_streams(st);
+    if (fork) {
+      // SM-seconds of each class at the rates one SM sustains on its own
+      const double a = prefill_flops / kPrefillFlopsPerSm;
+      const double b = (double)decode_keys * 2 * num_kv_heads * head_dim * 2 / kDecodeBytesPerSm;
+      prefill_ctas = (int)lround(sms * a / (a + b));
+      prefill_ctas = max(1, min(prefill_ctas, sms / 2));
+      decode_ctas = sms - prefill_ctas;
+    }
+  }
+  if (fork) {
+    if (cudaEventRecord(fork->start, st) != cudaSuccess ||
+        cudaStreamWaitEvent(fork->side, fork->start, 0) != cudaSuccess)
+      return PA_ERR_CUDA;
+    cudaError_t e = launch_prefill_tcgen05(p, head_dim, max_query_len, prefill_items,
+                                           seq_lens_host, query_start_loc_host, fork->side,
+                                           prefill_ctas);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    e = launch_decode(p, head_dim, seq_lens_host, query_start_loc_host, st, decode_ctas);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaEventRecord(fork->done, fork->side) != cudaSuccess ||
+        cudaStreamWaitEvent(st, fork->done, 0) != cudaSuccess)
+      return PA_ERR_CUDA;
+    return PA_OK;
+  }
   if (any_decode) {
-    cudaError_t e = launch_decode_splitk(p, head_dim, max_query_len, st);
+    cudaError_t e = launch_decode(p, head_dim, seq_lens_host, query_start_loc_host, st, sms);
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
   if (any_prefill) {
     cudaError_t e = launch_prefill_tcgen05(p, head_dim, max_query_len, prefill_items,
-                                           seq_lens_host, query_start_loc_host, st);
+                                           seq_lens_host, query_start_loc_host, st, sms);
     if (e != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
@@ -336,8 +410,29 @@ extern "C" int pa_attention_varlen(void* out, const void* q, const void* k_cache
                         query_start_loc, num_seqs, num_tokens, max_query_len, max_seq_len,
                         num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
                         workspace, workspace_bytes, seq_lens_host, query_start_loc_host, stream,
-                        CacheWrite{});
+                        CacheWrite{}, CallOptions{});
 }
+
+namespace pa {
+
+int attention_varlen_sequential(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* seq_lens, const int32_t* query_start_loc,
+                                int num_seqs, int num_tokens, int max_query_len, int max_seq_len,
+                                int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, float scale, pa_dtype dtype, void* workspace,
+                                size_t workspace_bytes, const int32_t* seq_lens_host,
+                                const int32_t* query_start_loc_host, struct CUstream_st* stream) {
+  CallOptions opt;
+  opt.allow_fork = false;
+  return attention_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, seq_lens,
+                        query_start_loc, num_seqs, num_tokens, max_query_len, max_seq_len,
+                        num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
+                        workspace, workspace_bytes, seq_lens_host, query_start_loc_host, stream,
+                        CacheWrite{}, opt);
+}
+
+}  // namespace pa
 
 extern "C" int pa_attention_varlen_write_cache(
     void* out, const void* q, const void* k_new, const void* v_new, void* k_cache,
@@ -356,5 +451,5 @@ extern "C" int pa_attention_varlen_write_cache(
                         query_start_loc, num_seqs, num_tokens, max_query_len, max_seq_len,
                         num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
                         workspace, workspace_bytes, seq_lens_host, query_start_loc_host, stream,
-                        slot_mapping ? cw : CacheWrite{});
+                        slot_mapping ? cw : CacheWrite{}, CallOptions{});
 }

@@ -8,6 +8,8 @@
 
 #include <atomic>
 
+#include "pa.h"
+
 namespace pa {
 
 // Raise a kernel's dynamic shared-memory limit only when a launch needs more
@@ -36,20 +38,33 @@ int device_sm_count();
 constexpr int kBlockSize = 16;       // tokens per cache block (the pages' default)
 constexpr int kDecodeRows = 16;      // query rows per kv-head one decode CTA holds (MMA M)
 // A decode-class sequence has at most kDecodeMaxRows query rows per kv-head
-// (q_len * q-heads per kv-head); they are split into 16-row groups, one CTA
-// each.  Longer queries are prefill chunks.
+// (q_len * q-heads per kv-head); they are split into 16-row groups, a unit of
+// decode work each.  Longer queries are prefill chunks.
 constexpr int kDecodeRowGroups = 4;
 constexpr int kDecodeMaxRows = kDecodeRows * kDecodeRowGroups;
-// split-K partitions per sequence the decode kernel can merge (its shared
-// memory holds each partition's per-row max and sum): 1536 partitions of at
-// least 1024 keys, i.e. sequences of at least 1.5M tokens
+// split-K partial slots the workspace holds per (sequence, kv-head), shared by
+// its row groups: kDecodePartsBase + ceil(max blocks / kDecodePartsPerBlocks)
+constexpr int kDecodePartsBase = 8;
+constexpr int kDecodePartsPerBlocks = 256;
+// sanity bound on the slots of one (sequence, kv-head)
 constexpr int kDecodeMaxParts = 1536;
-// sequences one decode launch covers (grid z)
-constexpr int kDecodeMaxSeqs = 65535;
-#ifndef PA_DECODE_WARPS
-#define PA_DECODE_WARPS 4
-#endif
-constexpr int kDecodeWarps = PA_DECODE_WARPS;  // warps of a decode CTA
+// pieces of decode work: blocks per piece, and pieces per CTA the launch aims at
+constexpr int kDecodeMaxPieceBlocks = 1024;
+constexpr int kDecodeMinPieceBlocks = 4;
+constexpr int kDecodePiecesPerCta = 4;
+// K+V bytes of one (block, kv-head) per piece at most, unless a long unit
+// needs bigger pieces to fit its partial slots
+constexpr long kDecodeMaxPieceBytes = 2l << 20;
+// pieces a launch can carry as a kernel parameter (more: the list is built on
+// the device, in the workspace); the parameter stays under 32 KB
+constexpr int kDecodeParamPieces = 1984;
+
+// words of the workspace header (the first 256 bytes)
+constexpr int kWsStatus = 0;       // error bits set by a kernel that gave up waiting
+constexpr int kWsClaim = 1;        // decode pieces claimed past the first one per CTA
+constexpr int kWsDone = 2;         // decode CTAs done claiming (the last resets both)
+constexpr int kWsPieceCount = 3;   // decode pieces in the device-built list
+constexpr int kWsPieceBlocks = 4;  // blocks per piece of that list
 
 // Everything one attention launch reads; the same struct serves every kernel.
 struct AttnParams {
@@ -70,26 +85,39 @@ struct AttnParams {
   int num_blocks;
   float scale;       // softmax scale (natural-log base)
   float scale_log2;  // scale * log2(e), for exp2-based softmax
-  // split-K decode
   // decode-class steps of pa_attention_varlen_write_cache: the new tokens' K/V
   // rows [num_tokens][Hkv][D] and their slots, written by the decode kernel
   // (null otherwise)
   const void* k_new;
   const void* v_new;
   const int64_t* slot_mapping;
-  int part_tokens;   // keys per partition at most (multiple of 16); a sequence is cut
-                     // into ceil(L / part_tokens) partitions of equal whole blocks
-  int max_parts;     // partial slots the workspace holds per (sequence, kv-head): one per
-                     // (partition, row group), partition-major
+  int max_parts;     // partial slots per (sequence, kv-head): one per (piece, row group),
+                     // piece-major
   int row_groups;    // 16-row groups per (sequence, kv-head) in this launch (1..4)
   int decode_rows;   // most query rows of one decode-class (sequence, kv-head)
+  int max_pieces;    // capacity of ws_pieces
   float* ws_o;       // [num_seqs*Hkv][max_parts][16][D] unnormalised partial outputs
   float* ws_ml;      // [num_seqs*Hkv][max_parts][16][2] running max (log2 units), sum
-  int* ws_counter;   // [num_seqs*Hkv] arrival counters, zero between calls
+  int* ws_counter;   // [num_seqs*Hkv][kDecodeRowGroups] arrival counters, zero between calls
+  int* ws_status;    // the workspace header (kWs* words); [0]: error bits
+  int* ws_header;    // = ws_status
+  int4* ws_pieces;   // device-built decode piece list
   // prefill work list
-  int* ws_status;    // [0]: error bits set by a kernel that gave up waiting
   int4* ws_items;    // prefill items (seq, q-tile, q-head, kv tiles)
   int max_items;
+};
+
+// A decode launch's piece list carried as a kernel parameter (from_ws = 0), or
+// a pointer to the device-built one in the workspace (from_ws = 1).  A piece is
+// one int4: x = sequence, y = q_len << 24 | row group << 22 | kv-head << 12 |
+// piece index in the unit, z = seq_len, w = query_start_loc of the sequence;
+// piece j of a unit covers blocks j * piece_blocks .. of its sequence.
+struct DecodeWork {
+  int count;
+  int piece_blocks;
+  int from_ws;
+  int pad;
+  int4 items[kDecodeParamPieces];
 };
 
 // bits of ws_status[0]
@@ -97,10 +125,10 @@ constexpr int kStatusWaitTimeout = 1;  // an mbarrier wait exceeded its time lim
 
 // Workspace layout shared by the size query and the launch.
 struct WorkspaceLayout {
-  int part_tokens;
   int max_parts;
   int max_items;
-  size_t status_off, counter_off, o_off, ml_off, items_off, total;
+  int max_pieces;
+  size_t status_off, counter_off, o_off, ml_off, pieces_off, items_off, total;
 };
 WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_seq_len);
@@ -116,22 +144,37 @@ cudaError_t launch_reshape_and_cache(const void* k, const void* v, void* k_cache
 cudaError_t launch_attention_simple(const AttnParams& p, int head_dim, bool is_bf16,
                                     int min_rows_per_kv_head, cudaStream_t stream);
 
-// Split-K decode kernel (bf16): sequences with q_len * group <= kDecodeMaxRows (64),
-// in 16-row groups.
-// Decode CTAs the GPU holds at once for this head_dim and query-row count
-// (SMs x resident CTAs per SM); looked up once per device and shape.
-int decode_wave_ctas(int head_dim, int rows);
-cudaError_t launch_decode_splitk(const AttnParams& p, int head_dim, int max_query_len,
-                                 cudaStream_t stream);
+// Persistent split-K decode kernel (bf16): sequences with q_len * group <=
+// kDecodeMaxRows (64), in 16-row groups.  With host copies of the lengths the
+// piece list is built on the host and passed with the launch; otherwise a
+// one-CTA planning kernel builds it in the workspace first.
+// At most max_ctas CTAs (the SMs left to decode when prefill runs beside it).
+cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_lens_host,
+                          const int32_t* query_start_loc_host, cudaStream_t stream,
+                          int max_ctas);
 
 // Tensor-core prefill kernel (bf16): sequences with q_len * group > kDecodeMaxRows.
 // num_items >= 0: the work list in ws_items was written by the host (exact
 // count); num_items < 0: build it on the device first.
 constexpr int kPrefillQTile = 128;  // query rows per Q tile (MMA M); a work item holds two
 constexpr int kPrefillKvTile = 128;  // keys per pipeline step
+// At most max_ctas persistent CTAs (one per SM).
 cudaError_t launch_prefill_tcgen05(const AttnParams& p, int head_dim, int max_query_len,
                                    int num_items, const int32_t* seq_lens_host,
-                                   const int32_t* query_start_loc_host, cudaStream_t stream);
+                                   const int32_t* query_start_loc_host, cudaStream_t stream,
+                                   int max_ctas);
+
+// pa_attention_varlen without the side stream of a mixed step (the two
+// classes run one after the other): for the caller that must not create any
+// CUDA object (the static-scratch entry point).
+int attention_varlen_sequential(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* seq_lens, const int32_t* query_start_loc,
+                                int num_seqs, int num_tokens, int max_query_len, int max_seq_len,
+                                int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, float scale, pa_dtype dtype, void* workspace,
+                                size_t workspace_bytes, const int32_t* seq_lens_host,
+                                const int32_t* query_start_loc_host, struct CUstream_st* stream);
 
 // On-GPU step planner (allocate_slots, seq_lens, query_start_loc, slot
 // mapping).  planner state: int32[4] in device memory.

@@ -16,7 +16,7 @@
 //   warp 8      TMA: the two Q tiles once per item, then every K tile -- eight
 //               16-token cache blocks, one 16 x 64 box per block and 64-wide
 //               slice of D, 128-byte swizzled, straight from the pool through
-//               the block table
+//               the block table; one lane issues each box
 //   warp 10     TMA: every V tile, the same way
 //   warp 9      MMA issuer (one thread): S_h = Q_h K^T into TMEM (tcgen05.mma,
 //               M=128, N=128, K=16 steps, both operands in shared memory), and
@@ -43,6 +43,7 @@
 
 #include "pa_fastmath.cuh"
 #include "pa_internal.cuh"
+#include "pa_wait.cuh"
 
 namespace pa {
 namespace {
@@ -71,12 +72,6 @@ constexpr uint32_t kTmemCols = 512;
 // TMEM columns: O of half h at 128 h; S of half h at 256 + 128 h, its P (bf16,
 // two per column) written over the first 64 columns of S once S is read
 constexpr uint32_t kTmemO = 0, kTmemS = 256;
-constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
-// longest single sleep of a waiting thread before it checks the limit again
-#ifndef PA_WAIT_SUSPEND_NS
-#define PA_WAIT_SUSPEND_NS 20000
-#endif
-constexpr uint32_t kWaitSuspendNs = PA_WAIT_SUSPEND_NS;
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: move the max only past 2^8
 // of every 8 pairs of score columns, how many take exp2 on the FMA pipe
 // (exp2_poly2) instead of the exponential unit
@@ -124,64 +119,6 @@ enum : int {
 static_assert(kNumBars * 8 <= 256, "barriers must fit their 256-byte area");
 
 // ------------------------------------------------------------------ PTX wrappers
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// The same, but a thread whose phase has not completed sleeps until it does,
-// or for at most suspend_ns, instead of returning at once: waiting warps then
-// take no issue slots from the warps that share their scheduler.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
-                                                    uint32_t suspend_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(suspend_ns)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase of `bar` with parity `parity` to complete.  Gives up
-// (returns false) when another role of the CTA has given up, or after the time
-// limit, in which case it records the timeout in the workspace status word.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait_sleep(bar, parity, kWaitSuspendNs)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      atomicOr(status, kStatusWaitTimeout);
-      return false;
-    }
-  }
-}
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, uint32_t bar) {
@@ -434,35 +371,32 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
         ok = __shfl_sync(0xffffffffu, ok, 0);
         // ---- K or V tiles
         for (int t = 0; t < it.ntiles && ok; ++t, ++g) {
+          // lane b < kTileBlocks reads the id of the tile's block b; lane
+          // pn * kTileBlocks + b then issues the box of block b, D-slice pn
           int id = -1;
           const int lb = t * kTileBlocks + lane;
           if (lane < kTileBlocks && lb < nblk && lb < p.max_blocks_per_seq) id = table[lb];
-          int c1[kTileBlocks], c2[kTileBlocks];
-  #pragma unroll
-          for (int b = 0; b < kTileBlocks; ++b) {
-            const int idb = __shfl_sync(0xffffffffu, id, b);
-            const int lbb = t * kTileBlocks + b;
-            const bool valid = lbb < nblk && idb >= 0 && idb < p.num_blocks;
-            c1[b] = (valid && lbb == nblk - 1) ? -shift : 0;
-            c2[b] = valid ? idb * p.num_kv_heads + kvh : oob_bh;
-          }
+          const int b = lane % kTileBlocks, pn = lane / kTileBlocks;
+          const int idb = __shfl_sync(0xffffffffu, id, b);
+          const int lbb = t * kTileBlocks + b;
+          const bool valid = lbb < nblk && idb >= 0 && idb < p.num_blocks;
+          const int c1 = (valid && lbb == nblk - 1) ? -shift : 0;
+          const int c2 = valid ? idb * p.num_kv_heads + kvh : oob_bh;
+          const uint32_t nst = is_v ? kVStages : kKStages;
+          const int st = g % nst;
+          const int full = (is_v ? kBarVFull : kBarKFull) + st;
+          const int empty = (is_v ? kBarVEmpty : kBarKEmpty) + st;
           if (lane == 0) {
-            const uint32_t nst = is_v ? kVStages : kKStages;
-            const int st = g % nst;
-            const int full = (is_v ? kBarVFull : kBarKFull) + st;
-            const int empty = (is_v ? kBarVEmpty : kBarKEmpty) + st;
-            const uint32_t dst = (is_v ? sV : sK) + st * LY::kKvBytes;
-            const CUtensorMap* map = is_v ? &tm_v : &tm_k;
             if (g >= nst) ok = wait_bar(bar(empty), ((g / nst) - 1) & 1, abort_flag, status);
-            if (ok) {
-              mbar_expect_tx(bar(full), LY::kKvBytes);
-              for (int pn = 0; pn < kPanels; ++pn)
-                for (int b = 0; b < kTileBlocks; ++b)
-                  tma_load_3d(dst + pn * LY::kKvPanelBytes + b * 2048, map, 64 * pn, c1[b], c2[b],
-                              bar(full));
-            }
+            if (ok) mbar_expect_tx(bar(full), LY::kKvBytes);
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = __shfl_sync(0xffffffffu, ok, 0);  // (also orders the expect_tx first)
+          if (ok && lane < kPanels * kTileBlocks) {
+            const uint32_t dst = (is_v ? sV : sK) + st * LY::kKvBytes;
+            tma_load_3d(dst + pn * LY::kKvPanelBytes + b * 2048, is_v ? &tm_v : &tm_k, 64 * pn,
+                        c1, c2, bar(full));
+          }
+          __syncwarp();
         }
       }
     } else if (warp == kWarpMma) {
@@ -864,7 +798,7 @@ bool host_work_list(PrefillWork* work, const AttnParams& p, const int32_t* seq_l
 template <int D>
 cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items,
                      const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, int max_ctas) {
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, p.q, D, p.num_q_heads, p.num_tokens, (uint64_t)D * 2,
                 (uint64_t)p.num_q_heads * D * 2, 1, QT) ||
@@ -909,7 +843,7 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items,
                                    : (int)min((long)p.max_items,
                                               (long)p.num_seqs * ((max_query_len + QT - 1) / QT) *
                                                   p.num_q_heads);
-  const int grid = max(1, min(device_sm_count(), upper));
+  const int grid = max(1, min(min(device_sm_count(), max_ctas), upper));
   auto kernel = prefill_tcgen05_kernel<D>;
   const int smem = PrefillLayout<D>::total;
   static std::atomic<int> smem_done[64];
@@ -929,12 +863,14 @@ cudaError_t launch_d(const AttnParams& p, int max_query_len, int num_items,
 
 cudaError_t launch_prefill_tcgen05(const AttnParams& p, int head_dim, int max_query_len,
                                    int num_items, const int32_t* seq_lens_host,
-                                   const int32_t* query_start_loc_host, cudaStream_t stream) {
+                                   const int32_t* query_start_loc_host, cudaStream_t stream,
+                                   int max_ctas) {
   cudaError_t e =
       head_dim == 64
-          ? launch_d<64>(p, max_query_len, num_items, seq_lens_host, query_start_loc_host, stream)
+          ? launch_d<64>(p, max_query_len, num_items, seq_lens_host, query_start_loc_host, stream,
+                         max_ctas)
           : launch_d<128>(p, max_query_len, num_items, seq_lens_host, query_start_loc_host,
-                          stream);
+                          stream, max_ctas);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

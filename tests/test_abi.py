@@ -73,12 +73,14 @@ def test_attention_argument_checks(L):
     assert _varlen(L, out=0) == palib.PA_ERR_INVALID
     assert _varlen(L, S=-1) == palib.PA_ERR_INVALID
     assert _varlen(L, T=0) == palib.PA_OK  # nothing to do, nothing launched
-    # more sequences than the decode grid holds (without host copies any
-    # sequence may be decode-class)
-    assert _varlen(L, S=65536, T=65536) == palib.PA_ERR_UNSUPPORTED
-    # a bound past what the split-K merge can hold (1537 partitions of 2048 keys)
-    assert _varlen(L, ms=1536 * 2048 + 1, mb=(1536 * 2048 + 1 + 15) // 16) == \
-        palib.PA_ERR_UNSUPPORTED
+    # any number of sequences: a large call is refused only for its missing
+    # workspace (the persistent decode grid does not depend on the count)
+    assert _varlen(L, S=65536, T=65536) == palib.PA_ERR_INVALID
+    # a bound past the split-K partial slots one (sequence, kv-head) may hold
+    # (8 + ceil(blocks / 256) > 1536)
+    big = 391_169 * 16
+    assert _varlen(L, ms=big, mb=big // 16) == palib.PA_ERR_UNSUPPORTED
+    assert _varlen(L, ms=big - 16, mb=big // 16) == palib.PA_ERR_INVALID  # fits, no workspace
     # host copies that contradict the scalars are rejected
     import numpy as np
     sl = np.array([4], np.int32)
@@ -152,6 +154,22 @@ def test_plan_step_argument_checks(L):
     assert _plan(L, slots=0) == palib.PA_ERR_INVALID     # room for 8 slots at NULL
     assert _plan(L, slots=20) == palib.PA_ERR_INVALID    # int64 slots misaligned
     assert _plan(L, ql=18) == palib.PA_ERR_INVALID       # int32 array misaligned
+
+
+def test_plan_step_rejects_outputs_aliasing_inputs(L):
+    """num_computed and query_lens are read in full by every CTA while other
+    CTAs write seq_lens, query_start_loc and the slots: a call whose outputs
+    share memory with those inputs is refused on the host."""
+    base = 1 << 20
+    ok = dict(nc=base, ql=base + 64, sl=base + 128, qsl=base + 192, slots=base + 256)
+    # the same pointers, but pa_plan_step never runs: a bad block size is
+    # reported first, so an otherwise valid set of separate buffers passes the
+    # alias check and fails only on the block size
+    assert _plan(L, bs=32, **ok) == palib.PA_ERR_UNSUPPORTED
+    assert _plan(L, **dict(ok, sl=ok["nc"])) == palib.PA_ERR_INVALID   # seq_lens = num_computed
+    assert _plan(L, **dict(ok, sl=ok["ql"] + 4)) == palib.PA_ERR_INVALID  # partly overlapping
+    assert _plan(L, **dict(ok, qsl=ok["nc"])) == palib.PA_ERR_INVALID
+    assert _plan(L, **dict(ok, slots=ok["ql"] - 8)) == palib.PA_ERR_INVALID
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
