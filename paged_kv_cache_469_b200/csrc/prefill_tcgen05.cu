@@ -73,12 +73,6 @@ constexpr uint32_t kTmemCols = 512;
 // two per column) written over the first 64 columns of S once S is read
 constexpr uint32_t kTmemO = 0, kTmemS = 256;
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: move the max only past 2^8
-// of every 8 pairs of score columns, how many take exp2 on the FMA pipe
-// (exp2_poly2) instead of the exponential unit
-#ifndef PA_PREFILL_POLY_PAIRS
-#define PA_PREFILL_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = PA_PREFILL_POLY_PAIRS;
 // independent max chains over a row of scores (a power of two, at most 32)
 #ifndef PA_PREFILL_MAX_CHAINS
 #define PA_PREFILL_MAX_CHAINS 8
@@ -559,10 +553,10 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           m_run = mx;
         }
         const float neg_base = (m_run == -INFINITY) ? 0.f : -m_run;
-        // ---- P = exp2(S * scale * log2(e) - max) on pairs of columns: kPolyPairs
-        // of every 8 pairs on the FMA pipe, the rest on the exponential unit;
-        // two bf16 per word, written over the first half of S in 32-word
-        // chunks (this thread has read all of S already)
+        // ---- P = exp2(S * scale * log2(e) - max) on pairs of columns (the
+        // scaling on the packed-pair FMA, the exponentials on the exponential
+        // unit); two bf16 per word, written over the first half of S in
+        // 32-word chunks (this thread has read all of S already)
         const uint64_t scale2 = f2(sl2, sl2), base2 = f2(neg_base, neg_base);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -572,14 +566,9 @@ prefill_tcgen05_kernel(const AttnParams p, const __grid_constant__ CUtensorMap t
           for (int j = 0; j < 32; ++j) {
             const int n = 64 * c + 2 * j;
             const uint64_t x = fma2(f2(s[n], s[n + 1]), scale2, base2);
-            uint64_t e;
-            if ((j & 7) < kPolyPairs) {
-              e = exp2_poly2(x);
-            } else {
-              float x0, x1;
-              f2_split(x, x0, x1);
-              e = f2(ex2(x0), ex2(x1));  // masked: ex2(-inf) = 0
-            }
+            float x0, x1;
+            f2_split(x, x0, x1);
+            const uint64_t e = f2(ex2(x0), ex2(x1));  // masked: ex2(-inf) = 0
             acc[j & 3] = add2(acc[j & 3], e);
             float e0, e1;
             f2_split(e, e0, e1);
