@@ -100,7 +100,9 @@ struct DecodeLayout {
   static constexpr int slot_off = (merge_end + 127) / 128 * 128;
   // per compute warp: (piece, block) of each ring stage
   static constexpr int meta_off = slot_off + 2 * kSlotBytes;
-  static constexpr int total = meta_off + kWarps * kStages * 8;
+  // per compute warp: per-row max and 1 / sum of a sequence's merged partials
+  static constexpr int msc_off = meta_off + kWarps * kStages * 8;
+  static constexpr int total = msc_off + kWarps * 2 * kMaxRows * 4;
   static_assert(sizeof(PieceInfo) <= kInfoBytes, "piece info");
   static_assert(kSlotBytes % 16 == 0, "piece slot alignment");
   static_assert(total <= 227 * 1024, "shared memory of one CTA");
@@ -210,6 +212,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   float* msl_l = reinterpret_cast<float*>(smem + LY::ml_off);
   float* msl_o = reinterpret_cast<float*>(smem + LY::mo_off);
   int* meta = reinterpret_cast<int*>(smem + LY::meta_off);  // [kWarps][kStages][2]
+  float* msc = reinterpret_cast<float*>(smem + LY::msc_off);  // [kWarps][2][kMaxRows]
   volatile int* vabort = &ctl.abort;
   int* status = p.ws_status;
 
@@ -465,14 +468,16 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     if (!last) return true;
     __threadfence_block();  // every lane sees the other warps' parts
 
-    // ---- merge the warps' parts of the piece
+    // ---- merge the warps' parts of the piece: shared memory in, global
+    // stores out, then the merge slot is free again (no round trip to global
+    // memory while the other warps may wait for the slot)
     const int nw = min(kWarps, inf->nb);
-    const int rows = inf->rows;
-    const int s = inf->s, kvh = inf->kvh, rg = inf->rg;
-    const int unit = s * p.num_kv_heads + kvh;
+    const int rows = inf->rows, row0 = inf->row0, q0 = inf->q0;
+    const int kvh = inf->kvh, rg = inf->rg, np = inf->nparts;
+    const int unit = inf->s * p.num_kv_heads + kvh;
     __nv_bfloat16* out = (__nv_bfloat16*)p.out;
     constexpr int D4 = D / 4;
-    const bool direct = inf->nparts == 1;
+    const bool direct = np == 1;
     const int64_t slot0 = ((int64_t)unit * p.max_parts + inf->j * p.row_groups + rg) * kDecodeRows;
     for (int e = lane; e < rows * D4; e += 32) {
       const int i = e / D4, d4 = e % D4;
@@ -488,8 +493,8 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
       }
       if (direct) {
-        const int gi = inf->row0 + i;
-        const int64_t tok = inf->q0 + gi / G, head = (int64_t)kvh * G + gi % G;
+        const int gi = row0 + i;
+        const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
         const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
         uint2 pk;
         pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
@@ -500,71 +505,98 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         if (d4 == 0) reinterpret_cast<float2*>(p.ws_ml)[slot0 + i] = make_float2(M, Ls);
       }
     }
-    if (!direct) {
-      // ---- the last arriving piece of the unit merges all of its partials
-      __threadfence();
-      __syncwarp();
-      int ulast = 0;
-      int* counter = p.ws_counter + unit * kDecodeRowGroups + rg;
-      if (lane == 0) ulast = atomicAdd(counter, 1) == inf->nparts - 1;
-      ulast = __shfl_sync(0xffffffffu, ulast, 0);
-      if (ulast) {
-        __threadfence();  // every lane sees the other pieces' partials
-        const int np = inf->nparts;
-        const int64_t uslot = ((int64_t)unit * p.max_parts + rg) * kDecodeRows;
-        const int64_t step = (int64_t)p.row_groups * kDecodeRows;  // next part, same row
-        const float2* pml = reinterpret_cast<const float2*>(p.ws_ml);
-        // per row: merged max and 1 / merged sum, kept in the (now read) merge slot
-        float* rM = msl_m;
-        float* rI = msl_l;
-        for (int i = 0; i < rows; ++i) {
-          float M = -INFINITY;
-          for (int q = lane; q < np; q += 32) M = fmaxf(M, __ldcg(pml + uslot + q * step + i).x);
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
-          const float base = (M == -INFINITY) ? 0.f : M;
-          float Ls = 0.f;
-          for (int q = lane; q < np; q += 32) {
-            const float2 ml = __ldcg(pml + uslot + q * step + i);
-            Ls += ml.y * exp2f(ml.x - base);
-          }
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o2);
-          if (lane == 0) {
-            rM[i] = base;
-            rI[i] = Ls > 0.f ? 1.f / Ls : 0.f;
-          }
-        }
-        __syncwarp();
-        const float4* po = reinterpret_cast<const float4*>(p.ws_o);
-        for (int e = lane; e < rows * D4; e += 32) {
-          const int i = e / D4, d4 = e % D4;
-          const float base = rM[i];
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-          for (int q = 0; q < np; ++q) {
-            const int64_t sl = uslot + q * step + i;
-            const float f = exp2f(__ldcg(pml + sl).x - base);
-            const float4 v = __ldcg(po + sl * D4 + d4);
-            acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
-          }
-          const float inv = rI[i];
-          const int gi = inf->row0 + i;
-          const int64_t tok = inf->q0 + gi / G, head = (int64_t)kvh * G + gi % G;
-          uint2 pk;
-          pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-          pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-          *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
-        }
-        if (lane == 0) *counter = 0;  // ready for the next call
-      }
-    }
-    __syncwarp();
+    __syncwarp();  // every lane is done with the merge slot and the piece slot
     if (lane == 0) {
       ctl.count = 0;
       __threadfence_block();
       *(volatile int*)&ctl.merged = pc;
     }
+    if (direct) return true;
+
+    // ---- the last arriving piece of the unit merges all of its partials
+    __threadfence();
+    __syncwarp();
+    int ulast = 0;
+    int* counter = p.ws_counter + unit * kDecodeRowGroups + rg;
+    if (lane == 0) ulast = atomicAdd(counter, 1) == np - 1;
+    ulast = __shfl_sync(0xffffffffu, ulast, 0);
+    if (!ulast) return true;
+    __threadfence();  // every lane sees the other pieces' partials
+    const int64_t uslot = ((int64_t)unit * p.max_parts + rg) * kDecodeRows;
+    const int64_t step = (int64_t)p.row_groups * kDecodeRows;  // the next part's same row
+    const float2* pml = reinterpret_cast<const float2*>(p.ws_ml);
+    const float4* po = reinterpret_cast<const float4*>(p.ws_o);
+    // per row: merged max and sum over the parts, 32 parts per round of loads
+    float Mr[kMaxRows], Lr[kMaxRows];
+#pragma unroll
+    for (int i = 0; i < kMaxRows; ++i) { Mr[i] = -INFINITY; Lr[i] = 0.f; }
+    for (int q0p = 0; q0p < np; q0p += 32) {
+      const int q = q0p + lane;
+      float2 ml[kMaxRows];
+#pragma unroll
+      for (int i = 0; i < kMaxRows; ++i)
+        ml[i] = (q < np && i < rows) ? __ldcg(pml + uslot + q * step + i)
+                                     : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int i = 0; i < kMaxRows; ++i) {
+        float m = ml[i].x;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o2));
+        const float Mn = fmaxf(Mr[i], m);
+        const float base = (Mn == -INFINITY) ? 0.f : Mn;
+        float l = ml[i].y * exp2f(ml[i].x - base);
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
+        Lr[i] = Lr[i] * exp2f(Mr[i] - base) + l;
+        Mr[i] = Mn;
+      }
+    }
+    float* wM = msc + warp * 2 * kMaxRows;  // this warp's scratch: per row max, 1 / sum
+    float* wI = wM + kMaxRows;
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < kMaxRows; ++i) {
+        wM[i] = (Mr[i] == -INFINITY) ? 0.f : Mr[i];
+        wI[i] = Lr[i] > 0.f ? 1.f / Lr[i] : 0.f;
+      }
+    }
+    __syncwarp();
+    // the output: (row, 4 dims) elements, four per lane per round of loads
+    constexpr int kE = kMaxRows * D4 / 32;
+    static_assert(kE * 32 == kMaxRows * D4, "elements per lane");
+#pragma unroll
+    for (int k0 = 0; k0 < kE; k0 += 4) {
+      float4 acc[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+      for (int q = 0; q < np; ++q) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = lane + 32 * (k0 + k), i = e / D4, d4 = e % D4;
+          if (k0 + k < kE && i < rows) {
+            const int64_t sl = uslot + q * step + i;
+            const float f = exp2f(__ldcg(pml + sl).x - wM[i]);
+            const float4 v = __ldcg(po + sl * D4 + d4);
+            acc[k].x += v.x * f; acc[k].y += v.y * f; acc[k].z += v.z * f; acc[k].w += v.w * f;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = lane + 32 * (k0 + k), i = e / D4, d4 = e % D4;
+        if (k0 + k < kE && i < rows) {
+          const float inv = wI[i];
+          const int gi = row0 + i;
+          const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
+          uint2 pk;
+          pk.x = pack_bf16x2(acc[k].x * inv, acc[k].y * inv);
+          pk.y = pack_bf16x2(acc[k].z * inv, acc[k].w * inv);
+          *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
+        }
+      }
+    }
+    if (lane == 0) *counter = 0;  // ready for the next call
     __syncwarp();
     return true;
   };
