@@ -92,11 +92,12 @@ int pa_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_ca
 
 /*
  * Bytes of workspace pa_attention_varlen needs for a step of at most
- * num_seqs sequences, no sequence longer than max_seq_len tokens: a status
- * word, fp32 split-K partials (running max, sum and unnormalised output per
- * partition of a sequence's keys), one int32 arrival counter per (sequence,
- * kv-head, 16-row group of query rows; four groups per kv-head) and the
- * prefill work list.  0 means invalid arguments.
+ * num_seqs sequences, no sequence longer than max_seq_len tokens: a 256-byte
+ * header (the status word, and counters the decode grid uses while it runs
+ * and leaves at zero), fp32 split-K partials (running max, sum and
+ * unnormalised output per piece of a sequence's keys), the decode work list
+ * when it is built on the device, and the prefill work list.  0 means
+ * invalid arguments.
  */
 size_t pa_attention_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                    int head_dim, int max_seq_len);

@@ -13,13 +13,17 @@
 // nblk cache blocks are cut into pieces of P blocks (the last one shorter).
 // The pieces of a launch form one list, largest first (every full piece, then
 // the shorter last pieces by falling size), so that the work still left at the
-// end of the launch is the finest.  P is chosen per launch from the step's
-// total blocks so that every CTA gets a few pieces.
+// end of the launch is the finest.  P is chosen per launch: when no unit is
+// much longer than a CTA's share of the step's blocks, every unit is one piece
+// (the largest-first claims balance the SMs and nothing needs merging across
+// CTAs); otherwise the long units are cut so that every CTA gets a few pieces.
 //
 // Grid.  One CTA per SM (its shared memory holds the streaming rings), each
-// running until the list is exhausted.  CTA b starts with piece b and then
-// claims further pieces from a global counter, one piece ahead of the one it
-// computes, so faster SMs take more pieces.  Inside a CTA:
+// running until the list is exhausted.  CTA b starts with piece b and claims
+// the next piece from a global counter once all blocks of its current piece
+// have been issued (their copies are still in flight while the claim and the
+// piece's staging complete), so the SMs that get through their work first
+// take the next pieces.  Inside a CTA:
 //
 //   scheduler warp (the last warp)  claims a piece, copies its block ids and
 //       its query rows into a shared-memory piece slot (two slots: piece p
@@ -36,10 +40,12 @@
 //         O[16 rows x D]      += P . V       D/8 mma.m16n8k16
 //   piece merge  when a warp has computed its last block of a piece it puts
 //       its (max, sum, O) in a shared merge slot; the last warp to arrive
-//       merges them and writes the piece's result: the output rows when the
-//       piece is the whole unit, else an fp32 partial in the workspace plus an
-//       arrival count per unit, the last arriving piece merging all partials
-//       of its unit into the output.  No CTA ever waits for another.
+//       merges them and stores the piece's result: the output rows when the
+//       piece is the whole unit, else an fp32 partial in the workspace.  No
+//       CTA ever waits for another, and no merge waits for global memory.
+//   combine kernel  (launched right after, as a programmatic dependent) one
+//       warp per unit cut into several pieces merges the unit's partials
+//       into its output rows.
 //
 // The dot product's D axis is permuted identically on Q and K so that every
 // lane's B-operand words are 8 consecutive bf16 of one key row, and the
@@ -100,9 +106,7 @@ struct DecodeLayout {
   static constexpr int slot_off = (merge_end + 127) / 128 * 128;
   // per compute warp: (piece, block) of each ring stage
   static constexpr int meta_off = slot_off + 2 * kSlotBytes;
-  // per compute warp: per-row max and 1 / sum of a sequence's merged partials
-  static constexpr int msc_off = meta_off + kWarps * kStages * 8;
-  static constexpr int total = msc_off + kWarps * 2 * kMaxRows * 4;
+  static constexpr int total = meta_off + kWarps * kStages * 8;
   static_assert(sizeof(PieceInfo) <= kInfoBytes, "piece info");
   static_assert(kSlotBytes % 16 == 0, "piece slot alignment");
   static_assert(total <= 227 * 1024, "shared memory of one CTA");
@@ -168,9 +172,10 @@ __device__ __forceinline__ int out_dim(int nt, int c) { return 64 * (nt / 8) + 8
 
 // Shared control words of a CTA.
 struct DecodeCtl {
-  int merged;  // CTA-local sequence number of the last piece merged (-1: none)
-  int count;   // compute warps that have put their part of the current piece in the merge slot
-  int abort;   // set by a bounded wait that ran out: every role winds down
+  int merged;     // CTA-local sequence number of the last piece merged (-1: none)
+  int count;      // compute warps that have put their part of the current piece in the merge slot
+  int abort;      // set by a bounded wait that ran out: every role winds down
+  int issued[2];  // blocks of the piece in each slot whose copies have been issued
 };
 
 // One piece of the list (see DecodeWork): x = sequence, y = ql << 24 | rg << 22
@@ -212,7 +217,6 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   float* msl_l = reinterpret_cast<float*>(smem + LY::ml_off);
   float* msl_o = reinterpret_cast<float*>(smem + LY::mo_off);
   int* meta = reinterpret_cast<int*>(smem + LY::meta_off);  // [kWarps][kStages][2]
-  float* msc = reinterpret_cast<float*>(smem + LY::msc_off);  // [kWarps][2][kMaxRows]
   volatile int* vabort = &ctl.abort;
   int* status = p.ws_status;
 
@@ -220,6 +224,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     ctl.merged = -1;
     ctl.count = 0;
     ctl.abort = 0;
+    ctl.issued[0] = ctl.issued[1] = 0;
     slot_info(0)->tag = -1;
     slot_info(1)->tag = -1;
   }
@@ -237,6 +242,16 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   if (warp == kWarps) {
     // =============================== scheduler ===============================
     for (int pc = 0;; ++pc) {
+      // the next piece is claimed only once every block of the current one
+      // has been issued (its copies then keep the warps busy for a while), so
+      // that the list's largest-first order goes to the SMs that are free
+      if (pc >= 1) {
+        const PieceInfo* prev = slot_info(pc - 1);
+        const int want = prev->nb;
+        if (!spin_until([&] { return *(volatile int*)&ctl.issued[(pc - 1) & 1] >= want; },
+                        vabort, status))
+          break;
+      }
       // slot pc % 2 is free once piece pc - 2 has been merged
       if (pc >= 2 &&
           !spin_until([&] { return *(volatile int*)&ctl.merged >= pc - 2; }, vabort, status))
@@ -324,6 +339,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         }
       }
       if (lane == 0) {
+        ctl.issued[pc & 1] = 0;
         inf->end = 0;
         inf->s = s; inf->kvh = kvh; inf->rg = rg; inf->j = j; inf->nparts = nparts;
         inf->blk_begin = blk_begin; inf->nb = nb;
@@ -415,6 +431,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     if (lane == 0) {
       my_meta[2 * st] = ip;
       my_meta[2 * st + 1] = ii;
+      atomicAdd(&ctl.issued[ip & 1], 1);
     }
     ++n_issued;
     ii += kWarps;
@@ -511,92 +528,6 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       __threadfence_block();
       *(volatile int*)&ctl.merged = pc;
     }
-    if (direct) return true;
-
-    // ---- the last arriving piece of the unit merges all of its partials
-    __threadfence();
-    __syncwarp();
-    int ulast = 0;
-    int* counter = p.ws_counter + unit * kDecodeRowGroups + rg;
-    if (lane == 0) ulast = atomicAdd(counter, 1) == np - 1;
-    ulast = __shfl_sync(0xffffffffu, ulast, 0);
-    if (!ulast) return true;
-    __threadfence();  // every lane sees the other pieces' partials
-    const int64_t uslot = ((int64_t)unit * p.max_parts + rg) * kDecodeRows;
-    const int64_t step = (int64_t)p.row_groups * kDecodeRows;  // the next part's same row
-    const float2* pml = reinterpret_cast<const float2*>(p.ws_ml);
-    const float4* po = reinterpret_cast<const float4*>(p.ws_o);
-    // per row: merged max and sum over the parts, 32 parts per round of loads
-    float Mr[kMaxRows], Lr[kMaxRows];
-#pragma unroll
-    for (int i = 0; i < kMaxRows; ++i) { Mr[i] = -INFINITY; Lr[i] = 0.f; }
-    for (int q0p = 0; q0p < np; q0p += 32) {
-      const int q = q0p + lane;
-      float2 ml[kMaxRows];
-#pragma unroll
-      for (int i = 0; i < kMaxRows; ++i)
-        ml[i] = (q < np && i < rows) ? __ldcg(pml + uslot + q * step + i)
-                                     : make_float2(-INFINITY, 0.f);
-#pragma unroll
-      for (int i = 0; i < kMaxRows; ++i) {
-        float m = ml[i].x;
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o2));
-        const float Mn = fmaxf(Mr[i], m);
-        const float base = (Mn == -INFINITY) ? 0.f : Mn;
-        float l = ml[i].y * exp2f(ml[i].x - base);
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
-        Lr[i] = Lr[i] * exp2f(Mr[i] - base) + l;
-        Mr[i] = Mn;
-      }
-    }
-    float* wM = msc + warp * 2 * kMaxRows;  // this warp's scratch: per row max, 1 / sum
-    float* wI = wM + kMaxRows;
-    if (lane == 0) {
-#pragma unroll
-      for (int i = 0; i < kMaxRows; ++i) {
-        wM[i] = (Mr[i] == -INFINITY) ? 0.f : Mr[i];
-        wI[i] = Lr[i] > 0.f ? 1.f / Lr[i] : 0.f;
-      }
-    }
-    __syncwarp();
-    // the output: (row, 4 dims) elements, four per lane per round of loads
-    constexpr int kE = kMaxRows * D4 / 32;
-    static_assert(kE * 32 == kMaxRows * D4, "elements per lane");
-#pragma unroll
-    for (int k0 = 0; k0 < kE; k0 += 4) {
-      float4 acc[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-      for (int q = 0; q < np; ++q) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int e = lane + 32 * (k0 + k), i = e / D4, d4 = e % D4;
-          if (k0 + k < kE && i < rows) {
-            const int64_t sl = uslot + q * step + i;
-            const float f = exp2f(__ldcg(pml + sl).x - wM[i]);
-            const float4 v = __ldcg(po + sl * D4 + d4);
-            acc[k].x += v.x * f; acc[k].y += v.y * f; acc[k].z += v.z * f; acc[k].w += v.w * f;
-          }
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int e = lane + 32 * (k0 + k), i = e / D4, d4 = e % D4;
-        if (k0 + k < kE && i < rows) {
-          const float inv = wI[i];
-          const int gi = row0 + i;
-          const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
-          uint2 pk;
-          pk.x = pack_bf16x2(acc[k].x * inv, acc[k].y * inv);
-          pk.y = pack_bf16x2(acc[k].z * inv, acc[k].w * inv);
-          *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
-        }
-      }
-    }
-    if (lane == 0) *counter = 0;  // ready for the next call
     __syncwarp();
     return true;
   };
@@ -792,6 +723,11 @@ __host__ __device__ __forceinline__ int decode_blocks(int ql, int L, int group, 
 __host__ __device__ __forceinline__ int choose_piece_blocks(long long total_blocks, int max_nblk,
                                                             int ctas, int slots_per_unit,
                                                             int head_dim) {
+  // Whole units when none is much longer than a CTA's share of the step: the
+  // largest-first claims then balance the SMs, and no unit needs a merge of
+  // partials across CTAs.
+  const long long share = total_blocks / max(1, ctas);
+  if (max_nblk <= kDecodeMaxPieceBlocks && 5ll * max_nblk <= 6 * share + 5 * 16) return max(1, max_nblk);
   long long want = (total_blocks + (long long)kDecodePiecesPerCta * ctas - 1) /
                    ((long long)kDecodePiecesPerCta * ctas);
   if (want < kDecodeMinPieceBlocks) want = kDecodeMinPieceBlocks;
@@ -944,7 +880,69 @@ bool host_piece_list(DecodeWork* work, const AttnParams& p, const int32_t* seq_l
   work->count = (int)run;
   work->piece_blocks = P;
   work->from_ws = 0;
+  work->split = mx > P;  // some unit has more than one piece
   return true;
+}
+
+// ------------------------------------------------------------------ combine
+
+// One warp per unit (sequence, kv-head, row group) whose blocks were cut into
+// more than one piece: merges the pieces' fp32 partials (running max, sum,
+// unnormalised O per row) into the output rows.  Launched as a programmatic
+// dependent of the decode kernel: it reads the partials only after that grid
+// has completed.
+template <int D>
+__global__ void __launch_bounds__(256)
+decode_combine_kernel(const AttnParams p, int piece_blocks, int from_ws) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const long u = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int RG = p.row_groups, G = p.group;
+  if (u >= (long)p.num_seqs * p.num_kv_heads * RG) return;
+  const int rg = (int)(u % RG);
+  const int kvh = (int)((u / RG) % p.num_kv_heads);
+  const int s = (int)(u / ((long)RG * p.num_kv_heads));
+  const int P = from_ws ? p.ws_header[kWsPieceBlocks] : piece_blocks;
+  const int q0 = p.query_start_loc[s], ql = p.query_start_loc[s + 1] - q0, L = p.seq_lens[s];
+  const int nblk = decode_blocks(ql, L, G, p.max_seq_len, p.max_blocks_per_seq);
+  if (!nblk || ql * G > p.decode_rows || P <= 0) return;
+  const int np = (nblk + P - 1) / P;
+  const int row0 = kDecodeRows * rg, rows = min(kDecodeRows, ql * G - row0);
+  if (np <= 1 || rows <= 0) return;
+  constexpr int D4 = D / 4;
+  const int64_t unit = (int64_t)s * p.num_kv_heads + kvh;
+  const int64_t uslot = (unit * p.max_parts + rg) * kDecodeRows;
+  const int64_t step = (int64_t)RG * kDecodeRows;  // the next part's same row
+  const float2* pml = reinterpret_cast<const float2*>(p.ws_ml);
+  const float4* po = reinterpret_cast<const float4*>(p.ws_o);
+  __nv_bfloat16* out = (__nv_bfloat16*)p.out;
+  // lane t handles (row, 4 dims) elements t, t + 32, ...; per element the max
+  // over the parts, then the weighted sums, the parts' loads issued together
+  for (int e = lane; e < rows * D4; e += 32) {
+    const int i = e / D4, d4 = e % D4;
+    float M = -INFINITY;
+    for (int q = 0; q < np; ++q) M = fmaxf(M, __ldcg(pml + uslot + q * step + i).x);
+    const float base = (M == -INFINITY) ? 0.f : M;
+    float Ls = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int q = 0; q < np; ++q) {
+      const int64_t sl = uslot + q * step + i;
+      const float2 ml = __ldcg(pml + sl);
+      const float f = exp2f(ml.x - base);
+      const float4 v = __ldcg(po + sl * D4 + d4);
+      Ls += ml.y * f;
+      acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+    }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    const int gi = row0 + i;
+    const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
+  }
 }
 
 template <int D, int kMaxRows>
@@ -994,6 +992,7 @@ cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_
     work.count = 0;
     work.piece_blocks = 0;
     work.from_ws = 1;
+    work.split = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(1024);
@@ -1015,6 +1014,24 @@ cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_
     e = wc ? launch_rows<128, true>(p, work, grid, max_rows, stream)
            : launch_rows<128, false>(p, work, grid, max_rows, stream);
   if (e != cudaSuccess) return e;
+  if (work.from_ws || work.split) {
+    // the units cut into several pieces: merge their partials
+    const long units = (long)p.num_seqs * p.num_kv_heads * p.row_groups;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((units + 7) / 8));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = head_dim == 64
+            ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, p, work.piece_blocks, work.from_ws)
+            : cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, p, work.piece_blocks,
+                                 work.from_ws);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 

@@ -44,10 +44,8 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads
   // the device-built piece list: at most one piece per partial slot
   w.max_pieces = (int)min(units * (size_t)w.max_parts, (size_t)(1 << 30));
   const size_t slots = units * w.max_parts * kDecodeRows;
-  w.status_off = 0;
-  w.counter_off = 256;
-  // one arrival counter per (sequence, kv-head, row group)
-  w.o_off = align_up(w.counter_off + units * kDecodeRowGroups * sizeof(int), 256);
+  w.status_off = 0;  // the 256-byte header: status word and the decode grid's counters
+  w.o_off = 256;
   w.ml_off = align_up(w.o_off + slots * head_dim * sizeof(float), 256);
   w.pieces_off = align_up(w.ml_off + slots * 2 * sizeof(float), 256);
   w.items_off = align_up(w.pieces_off + (size_t)w.max_pieces * 16, 256);
@@ -338,7 +336,6 @@ int attention_impl(void* out, const void* q, const void* k_cache, const void* v_
   char* ws = (char*)workspace;
   p.ws_status = (int*)(ws + w.status_off);
   p.ws_header = p.ws_status;
-  p.ws_counter = (int*)(ws + w.counter_off);
   p.ws_o = (float*)(ws + w.o_off);
   p.ws_ml = (float*)(ws + w.ml_off);
   p.ws_pieces = (int4*)(ws + w.pieces_off);

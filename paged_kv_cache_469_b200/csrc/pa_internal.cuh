@@ -98,7 +98,6 @@ struct AttnParams {
   int max_pieces;    // capacity of ws_pieces
   float* ws_o;       // [num_seqs*Hkv][max_parts][16][D] unnormalised partial outputs
   float* ws_ml;      // [num_seqs*Hkv][max_parts][16][2] running max (log2 units), sum
-  int* ws_counter;   // [num_seqs*Hkv][kDecodeRowGroups] arrival counters, zero between calls
   int* ws_status;    // the workspace header (kWs* words); [0]: error bits
   int* ws_header;    // = ws_status
   int4* ws_pieces;   // device-built decode piece list
@@ -116,7 +115,7 @@ struct DecodeWork {
   int count;
   int piece_blocks;
   int from_ws;
-  int pad;
+  int split;  // some unit has more than one piece (its partials need the combine kernel)
   int4 items[kDecodeParamPieces];
 };
 
@@ -128,7 +127,7 @@ struct WorkspaceLayout {
   int max_parts;
   int max_items;
   int max_pieces;
-  size_t status_off, counter_off, o_off, ml_off, pieces_off, items_off, total;
+  size_t status_off, o_off, ml_off, pieces_off, items_off, total;
 };
 WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int max_seq_len);

@@ -109,10 +109,11 @@ def test_static_scratch_against_the_oracle():
 
 
 def test_static_scratch_smaller_layout_after_larger_split_k():
-    """A many-partition split-K step fills the array's counters and partials
-    under a large layout; a smaller step with split-K sequences of its own
-    follows, without host copies (so its plan is estimated), and must still
-    be right: the counters it uses lie where the larger layout kept partials."""
+    """A step whose sequences are cut into many pieces fills the array's
+    partials and decode work list under a large layout; a smaller step with
+    pieces of its own follows, without host copies (so its work list is built
+    on the device), and must still be right: its header words and lists lie
+    where the larger layout kept other data."""
     from paged_kv_cache_469_b200.step import DeviceStep
     f = _entry()
     big = make_step(name="big", dtype="bf16", num_q_heads=32, num_kv_heads=8, head_dim=128,
