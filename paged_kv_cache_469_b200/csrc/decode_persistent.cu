@@ -62,6 +62,7 @@
 #include <math.h>
 
 #include "pa_internal.cuh"
+#include "pa_tma.cuh"
 #include "pa_wait.cuh"
 
 namespace pa {
@@ -69,9 +70,15 @@ namespace {
 
 // compute warps and ring stages per CTA, by head_dim and most query rows per
 // unit (shared memory: ring + merge slot + two piece slots, at most 227 KB)
+// A warp's loop over its blocks is bound by the latency of its own dependent
+// chain (loads, MMAs, shuffles, exponentials), about 2,000 cycles per block,
+// so an SM needs about a dozen compute warps to keep up with its share of
+// HBM bandwidth; the register budget of a quarter-SM (16K registers) and the
+// shared memory of the rings set how many fit.
 template <int D, int kMaxRows>
 struct DecodeCfg {
-  static constexpr int kWarps = D == 64 ? 8 : (kMaxRows <= 4 ? 8 : kMaxRows <= 8 ? 7 : 6);
+  static constexpr int kWarps =
+      D == 64 ? (kMaxRows <= 8 ? 11 : 8) : (kMaxRows <= 4 ? 8 : kMaxRows <= 8 ? 7 : 6);
   static constexpr int kStages = D == 64 ? 4 : 3;
 };
 
@@ -91,7 +98,7 @@ struct DecodeLayout {
   static constexpr int kStages = DecodeCfg<D, kMaxRows>::kStages;
   static constexpr int kTileBytes = kBlockSize * D * 2;  // one (block, kv-head) tile
   static constexpr int kStageBytes = 2 * kTileBytes;     // K tile + V tile
-  static constexpr int ring_off = 0;
+  static constexpr int ring_off = 0;  // 1024-byte aligned (128-byte swizzle atoms)
   static constexpr int ring_bytes = kWarps * kStages * kStageBytes;
   // merge slot: per compute warp its rows' max, sum and unnormalised O
   static constexpr int mm_off = ring_off + ring_bytes;                // [kWarps][kMaxRows]
@@ -106,7 +113,10 @@ struct DecodeLayout {
   static constexpr int slot_off = (merge_end + 127) / 128 * 128;
   // per compute warp: (piece, block) of each ring stage
   static constexpr int meta_off = slot_off + 2 * kSlotBytes;
-  static constexpr int total = meta_off + kWarps * kStages * 8;
+  // per compute warp and stage: the mbarrier its TMA loads complete on
+  static constexpr int bar_off = meta_off + kWarps * kStages * 8;
+  // (+1024: the dynamic shared memory base is rounded up to 1024 bytes)
+  static constexpr int total = bar_off + kWarps * kStages * 8 + 1024;
   static_assert(sizeof(PieceInfo) <= kInfoBytes, "piece info");
   static_assert(kSlotBytes % 16 == 0, "piece slot alignment");
   static_assert(total <= 227 * 1024, "shared memory of one CTA");
@@ -125,27 +135,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t smem, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-// wait until at most `pending` of this thread's newest copy groups are in flight
-template <int kStages>
-__device__ __forceinline__ void cp_async_wait_pending(int pending) {
-  static_assert(kStages <= 5, "cp_async_wait_pending");
-  if (pending <= 0) cp_async_wait<0>();
-  else if (pending == 1) cp_async_wait<1>();
-  else if (pending == 2) cp_async_wait<2>();
-  else if (pending == 3) cp_async_wait<3>();
-  else cp_async_wait<4>();
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
@@ -158,12 +147,37 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// XOR applied to the 16-byte chunk index of tile row `row` (K and V tiles).
-// K rows are read two at a time (rows 2k, 2k+1, chunk 4j..4j+3): flip the
-// half of the 128-byte line on odd rows.  V rows are read four at a time
-// (rows of equal parity), one chunk each: spread them by row bits 1-2.
-__device__ __forceinline__ int k_swz(int row) { return (row & 1) << 2; }
-__device__ __forceinline__ int v_swz(int row) { return row & 6; }
+// CTA-scope hand-offs in shared memory: release stores, acquire loads and
+// acq_rel adds order the memory accesses around them without a full fence
+// (a fence could also wait for the warp's copies still in flight).
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v)
+               : "r"((uint32_t)__cvta_generic_to_shared(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(p)),
+               "r"(v) : "memory");
+}
+__device__ __forceinline__ int add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old)
+               : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(v) : "memory");
+  return old;
+}
+
+// Byte offset of 16-byte chunk c of row `row` in a tile that TMA loaded as
+// 16 x 64 boxes with 128-byte swizzle: box (64-wide slice of D) c / 8 at
+// 2048 bytes per box, rows of 128 bytes, chunk c % 8 XOR row % 8.
+__device__ __forceinline__ uint32_t swz128(int row, int c) {
+  return (uint32_t)((c >> 3) * 2048 + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
+// 16-byte chunk of a key row (and of a query row) that lane q4 holds for the
+// jp-th pair of Q.K^T MMAs: the dot product's D axis is permuted so that the
+// eight lanes of one shared-memory phase (two rows, four q4) read eight
+// distinct banks after the swizzle (rows r and r+1 differ in row % 8 bit 0).
+__device__ __forceinline__ int k_chunk(int q4, int jp) { return 8 * (jp >> 1) + 2 * q4 + (jp & 1); }
 
 // Output column c (0..7) of n-tile nt sits at dimension 64*(nt/8) + 8*c + nt%8,
 // so a lane owning columns 2*q4, 2*q4+1 of every n-tile owns, per 64-wide
@@ -175,7 +189,7 @@ struct DecodeCtl {
   int merged;     // CTA-local sequence number of the last piece merged (-1: none)
   int count;      // compute warps that have put their part of the current piece in the merge slot
   int abort;      // set by a bounded wait that ran out: every role winds down
-  int issued[2];  // blocks of the piece in each slot whose copies have been issued
+  int passed[2];  // compute warps whose issue cursor has left the piece in each slot
 };
 
 // One piece of the list (see DecodeWork): x = sequence, y = ql << 24 | rg << 22
@@ -186,7 +200,9 @@ __device__ __forceinline__ int4 load_piece(const AttnParams& p, const DecodeWork
 
 template <int D, int kMaxRows, bool kWriteCache>
 __global__ void __launch_bounds__((DecodeCfg<D, kMaxRows>::kWarps + 1) * 32, 1)
-decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork work) {
+decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork work,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v) {
   using LY = DecodeLayout<D, kMaxRows>;
   constexpr int kWarps = LY::kWarps;
   constexpr int kStages = LY::kStages;
@@ -195,14 +211,16 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   constexpr int NV = D / 64;  // 16-byte V chunks per key row a lane reads
   constexpr int NT = D / 8;   // n-tiles of the P.V product
   constexpr int NC = D / 16;  // k-chunks of the Q.K^T product
-  constexpr int kChunks = D / 8;                        // 16-byte chunks per tile row
-  constexpr int kCopies = kBlockSize * kChunks / 32;    // 16-byte copies per lane per tile
+  constexpr int kChunks = D / 8;    // 16-byte chunks per tile row
+  constexpr int kPanels = D / 64;   // 64-wide slices of D: one 16 x 64 TMA box each
 
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ DecodeCtl ctl;
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+  const uint32_t sraw = (uint32_t)__cvta_generic_to_shared(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (sbase - sraw);
   auto slot_info = [&](int p_) {
     return reinterpret_cast<PieceInfo*>(smem + LY::slot_off + (p_ & 1) * LY::kSlotBytes);
   };
@@ -217,6 +235,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   float* msl_l = reinterpret_cast<float*>(smem + LY::ml_off);
   float* msl_o = reinterpret_cast<float*>(smem + LY::mo_off);
   int* meta = reinterpret_cast<int*>(smem + LY::meta_off);  // [kWarps][kStages][2]
+  const uint32_t bars = sbase + LY::bar_off;                 // [kWarps][kStages] mbarriers
   volatile int* vabort = &ctl.abort;
   int* status = p.ws_status;
 
@@ -224,9 +243,13 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     ctl.merged = -1;
     ctl.count = 0;
     ctl.abort = 0;
-    ctl.issued[0] = ctl.issued[1] = 0;
+    ctl.passed[0] = ctl.passed[1] = 0;
     slot_info(0)->tag = -1;
     slot_info(1)->tag = -1;
+    for (int i = 0; i < kWarps * kStages; ++i) mbar_init(bars + 8 * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
   }
   __syncthreads();
   // Launched as a programmatic dependent: nothing the preceding kernel may
@@ -243,18 +266,16 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     // =============================== scheduler ===============================
     for (int pc = 0;; ++pc) {
       // the next piece is claimed only once every block of the current one
-      // has been issued (its copies then keep the warps busy for a while), so
-      // that the list's largest-first order goes to the SMs that are free
-      if (pc >= 1) {
-        const PieceInfo* prev = slot_info(pc - 1);
-        const int want = prev->nb;
-        if (!spin_until([&] { return *(volatile int*)&ctl.issued[(pc - 1) & 1] >= want; },
-                        vabort, status))
-          break;
-      }
+      // has been issued (every compute warp's issue cursor has left it; the
+      // copies then keep the warps busy for a while), so that the list's
+      // largest-first order goes to the SMs that are free
+      if (pc >= 1 &&
+          !spin_until([&] { return ld_acquire(&ctl.passed[(pc - 1) & 1]) >= kWarps; }, vabort,
+                      status))
+        break;
       // slot pc % 2 is free once piece pc - 2 has been merged
       if (pc >= 2 &&
-          !spin_until([&] { return *(volatile int*)&ctl.merged >= pc - 2; }, vabort, status))
+          !spin_until([&] { return ld_acquire(&ctl.merged) >= pc - 2; }, vabort, status))
         break;
       int g = blockIdx.x;
       if (pc > 0) {
@@ -265,8 +286,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       if (g >= num_pieces) {
         if (lane == 0) {
           inf->end = 1;
-          __threadfence_block();
-          *(volatile int*)&inf->tag = pc;
+          st_release(&inf->tag, pc);
         }
         break;
       }
@@ -282,25 +302,49 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       const int rows_all = ql * G;
       const int row0 = kDecodeRows * rg;
       const int rows = min(kDecodeRows, rows_all - row0);
-      // block ids
+      // block ids and query rows (rows past the unit's are zero): every load
+      // of a round is issued before its results are stored, so that a piece
+      // is staged in one round trip to global memory (two for long pieces)
       const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks_per_seq + blk_begin;
       int* ids = slot_ids(pc);
-      for (int i = lane; i < nb; i += 32) ids[i] = table[i];
-      // query rows (rows past the unit's are zero)
+      constexpr int kQv = (kMaxRows * kChunks + 31) / 32;  // 16-byte query loads per lane
       {
         const uint4* qg = (const uint4*)p.q;
-        const uint32_t qs = slot_q(pc);
-        for (int c = lane; c < kMaxRows * kChunks; c += 32) {
-          const int i = c / kChunks, ch = c % kChunks;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (i < rows) {
+        uint4 qv[kQv];
+        int iv[8];
+#pragma unroll
+        for (int k = 0; k < kQv; ++k) {
+          const int c = lane + 32 * k, i = c / kChunks, ch = c % kChunks;
+          qv[k] = make_uint4(0, 0, 0, 0);
+          if (c < kMaxRows * kChunks && i < rows) {
             const int gi = row0 + i;
             const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
-            v = qg[(tok * p.num_q_heads + head) * kChunks + ch];
+            qv[k] = qg[(tok * p.num_q_heads + head) * kChunks + ch];
           }
-          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(qs + c * 16), "r"(v.x),
-                       "r"(v.y), "r"(v.z), "r"(v.w)
-                       : "memory");
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) iv[k] = lane + 32 * k < nb ? table[lane + 32 * k] : 0;
+        const uint32_t qs = slot_q(pc);
+#pragma unroll
+        for (int k = 0; k < kQv; ++k) {
+          const int c = lane + 32 * k;
+          if (c < kMaxRows * kChunks)
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(qs + c * 16),
+                         "r"(qv[k].x), "r"(qv[k].y), "r"(qv[k].z), "r"(qv[k].w)
+                         : "memory");
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (lane + 32 * k < nb) ids[lane + 32 * k] = iv[k];
+        for (int base = 256; base < nb; base += 256) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int i = base + lane + 32 * k;
+            iv[k] = i < nb ? table[i] : 0;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (base + lane + 32 * k < nb) ids[base + lane + 32 * k] = iv[k];
         }
       }
       if constexpr (kWriteCache) {
@@ -335,11 +379,13 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
             if (is_v) vcw[dst] = vn[src];
             else kcw[dst] = kn[src];
           }
+          // the compute warps read these rows with TMA (the async proxy)
           __threadfence();
+          asm volatile("fence.proxy.async.global;" ::: "memory");
         }
       }
       if (lane == 0) {
-        ctl.issued[pc & 1] = 0;
+        ctl.passed[pc & 1] = 0;
         inf->end = 0;
         inf->s = s; inf->kvh = kvh; inf->rg = rg; inf->j = j; inf->nparts = nparts;
         inf->blk_begin = blk_begin; inf->nb = nb;
@@ -347,10 +393,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         inf->rows = rows; inf->row0 = row0;
       }
       __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        *(volatile int*)&inf->tag = pc;
-      }
+      if (lane == 0) st_release(&inf->tag, pc);
     }
     // the last CTA to finish claiming resets the claim counter for the next call
     if (lane == 0) {
@@ -366,17 +409,18 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
 
   // ================================ compute warps ================================
   const int r = lane >> 2, q4 = lane & 3;
-  const char* kc = (const char*)p.k_cache;
-  const char* vc = (const char*)p.v_cache;
-  const int64_t blk_bytes = (int64_t)LY::kTileBytes * p.num_kv_heads;
+  const int oob_bh = p.num_blocks * p.num_kv_heads;  // first (block, kv-head) row past the pool
   const uint32_t ring = sbase + LY::ring_off + warp * kStages * LY::kStageBytes;
   int* my_meta = meta + warp * kStages * 2;
 
-  // the piece in slot pc, once published (nullptr before)
+  // the piece in slot pc, once published (nullptr before); the tag is read
+  // (with acquire order) only until the warp has seen the piece published
+  int seen = -1;  // the latest piece this warp has seen published
   auto published = [&](int pc) -> const PieceInfo* {
     const PieceInfo* inf = slot_info(pc);
-    if (*(volatile const int*)&inf->tag != pc) return nullptr;
-    __threadfence_block();
+    if (pc <= seen) return inf;
+    if (ld_acquire(&inf->tag) != pc) return nullptr;
+    seen = pc;
     return inf;
   };
 
@@ -404,34 +448,33 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         return false;
       }
       if (ii < inf->nb) break;
+      if (lane == 0) atomicAdd(&ctl.passed[ip & 1], 1);  // this warp leaves piece ip
       ++ip;
       ii = warp;
     }
     const int st = n_issued % kStages;
-    int id = slot_ids(ip)[ii];
-    if (id < 0 || id >= p.num_blocks) {  // never dereference outside the pool
-      id = 0;
-      bad |= 1u << st;
-    } else {
-      bad &= ~(1u << st);
-    }
-    const int64_t off = (int64_t)id * blk_bytes + (int64_t)LY::kTileBytes * inf->kvh;
-    const char* kt = kc + off;
-    const char* vt = vc + off;
-    const uint32_t ks = ring + st * LY::kStageBytes;
-    const uint32_t vs = ks + LY::kTileBytes;
+    const int id = slot_ids(ip)[ii];
+    // a block id outside the pool is never dereferenced: the box is read from
+    // past the tensor's extent (zeros) and its keys are masked
+    const bool id_ok = id >= 0 && id < p.num_blocks;
+    if (id_ok) bad &= ~(1u << st);
+    else bad |= 1u << st;
+    const int row_bh = id_ok ? id * p.num_kv_heads + inf->kvh : oob_bh;
+    if (lane == 0) {
+      const uint32_t ks = ring + st * LY::kStageBytes;
+      const uint32_t bar = bars + 8 * (warp * kStages + st);
+      // (the warp's earlier reads of this stage have completed: their values
+      // went into MMAs before the stage was freed)
+      mbar_expect_tx(bar, LY::kStageBytes);
 #pragma unroll
-    for (int c = 0; c < kCopies; ++c) {
-      const int idx = lane + 32 * c;
-      const int row = idx / kChunks, ch = idx % kChunks;
-      cp_async16(ks + (row * kChunks + (ch ^ k_swz(row))) * 16, kt + idx * 16);
-      cp_async16(vs + (row * kChunks + (ch ^ v_swz(row))) * 16, vt + idx * 16);
+      for (int pn = 0; pn < kPanels; ++pn) {
+        tma_load_3d(ks + pn * 2048, &tm_k, 64 * pn, 0, row_bh, bar);
+        tma_load_3d(ks + LY::kTileBytes + pn * 2048, &tm_v, 64 * pn, 0, row_bh, bar);
+      }
     }
-    cp_async_commit();
     if (lane == 0) {
       my_meta[2 * st] = ip;
       my_meta[2 * st + 1] = ii;
-      atomicAdd(&ctl.issued[ip & 1], 1);
     }
     ++n_issued;
     ii += kWarps;
@@ -455,7 +498,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
     }
     // the merge slot holds one piece at a time: the previous one must be merged
-    if (!spin_until([&] { return *(volatile int*)&ctl.merged >= pc - 1; }, vabort, status))
+    if (!spin_until([&] { return ld_acquire(&ctl.merged) >= pc - 1; }, vabort, status))
       return false;
     if (q4 == 0) {
       if (r < kMaxRows) { msl_m[warp * kMaxRows + r] = m_a; msl_l[warp * kMaxRows + r] = l_a; }
@@ -476,14 +519,10 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     }
     __syncwarp();
     int last = 0;
-    if (lane == 0) {
-      __threadfence_block();
-      const int arrived = atomicAdd(&ctl.count, 1) + 1;
-      last = arrived == min(kWarps, inf->nb);
-    }
+    if (lane == 0) last = add_acq_rel(&ctl.count, 1) + 1 == min(kWarps, inf->nb);
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return true;
-    __threadfence_block();  // every lane sees the other warps' parts
+    __syncwarp();  // every lane reads the other warps' parts after lane 0's acquire
 
     // ---- merge the warps' parts of the piece: shared memory in, global
     // stores out, then the merge slot is free again (no round trip to global
@@ -498,16 +537,26 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     const int64_t slot0 = ((int64_t)unit * p.max_parts + inf->j * p.row_groups + rg) * kDecodeRows;
     for (int e = lane; e < rows * D4; e += 32) {
       const int i = e / D4, d4 = e % D4;
+      // every warp's value loaded first (unrolled over the CTA's warps), then
+      // the max and the weighted sums
+      float mw[kWarps];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) mw[w] = w < nw ? msl_m[w * kMaxRows + i] : -INFINITY;
       float M = -INFINITY;
-      for (int w = 0; w < nw; ++w) M = fmaxf(M, msl_m[w * kMaxRows + i]);
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mw[w]);
       const float base = (M == -INFINITY) ? 0.f : M;
       float Ls = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int w = 0; w < nw; ++w) {
-        const float f = exp2f(msl_m[w * kMaxRows + i] - base);
-        Ls += msl_l[w * kMaxRows + i] * f;
-        const float4 v = *reinterpret_cast<const float4*>(msl_o + (w * kMaxRows + i) * D + 4 * d4);
-        acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        if (w < nw) {
+          const float f = exp2f(mw[w] - base);
+          Ls += msl_l[w * kMaxRows + i] * f;
+          const float4 v =
+              *reinterpret_cast<const float4*>(msl_o + (w * kMaxRows + i) * D + 4 * d4);
+          acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+        }
       }
       if (direct) {
         const int gi = row0 + i;
@@ -525,22 +574,69 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     __syncwarp();  // every lane is done with the merge slot and the piece slot
     if (lane == 0) {
       ctl.count = 0;
-      __threadfence_block();
-      *(volatile int*)&ctl.merged = pc;
+      st_release(&ctl.merged, pc);
     }
     __syncwarp();
     return true;
   };
 
+  // The loop is software-pipelined by one block: iteration n computes
+  // S = Q K^T and P of block n (phase A) and adds P V of block n-1 (phase B),
+  // two independent dependency chains; O is then rescaled to block n's
+  // running max.  A block whose P.V is still pending keeps its stage.  The
+  // warp's last block of a piece finishes at once, before the piece is
+  // flushed, so nothing is pending across pieces.
+  bool pend = false;
+  int pend_st = 0, pend_blk = 0, pend_L = 0;
+  bool pend_ok = true;
+  uint32_t pp0 = 0u, pp1 = 0u, pp2 = 0u, pp3 = 0u;  // P of the pending block, bf16 pairs
+  int n_done = 0;  // blocks whose stage is free again (their P.V is in O)
+
+  auto phase_b = [&]() {  // O += P V of the pending block
+    const uint32_t vs = ring + pend_st * LY::kStageBytes + LY::kTileBytes;
+    // V words: keys 2q4, 2q4+1, 2q4+8, 2q4+9; 8 dims 64u+8r.. each
+    uint4 vw[4][NV];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = 2 * q4 + (e & 1) + 8 * (e >> 1);
+#pragma unroll
+      for (int u = 0; u < NV; ++u) vw[e][u] = lds128(vs + swz128(tok, 8 * u + r));
+    }
+    // slots of the last block past seq_len (and blocks outside the pool) may
+    // hold anything, NaN included: their V words become zeros so that the
+    // zero weights cannot turn them into NaN in the P.V product
+    if (pend_blk * kBlockSize + kBlockSize > pend_L || !pend_ok) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = pend_blk * kBlockSize + 2 * q4 + (e & 1) + 8 * (e >> 1);
+        if (!pend_ok || key >= pend_L) {
+#pragma unroll
+          for (int u = 0; u < NV; ++u) vw[e][u] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int u = nt / 8, idx = nt % 8;
+      const uint32_t sel = (idx & 1) ? 0x7632u : 0x5410u;
+      const uint32_t b0 = __byte_perm(word(vw[0][u], idx >> 1), word(vw[1][u], idx >> 1), sel);
+      const uint32_t b1 = __byte_perm(word(vw[2][u], idx >> 1), word(vw[3][u], idx >> 1), sel);
+      mma_16816(o[nt], pp0, pp1, pp2, pp3, b0, b1);
+    }
+    pend = false;
+    ++n_done;
+  };
+
   while (true) {
-    // keep kStages blocks in flight; wait for a piece to be published only
-    // when nothing is in flight
-    while (!issue_done && n_issued - n_comp < kStages) {
-      if (!try_issue(n_issued == n_comp)) break;
+    // keep kStages blocks in flight (a pending block's stage included); wait
+    // for a piece to be published only when nothing is in flight
+    while (!issue_done && n_issued - n_done < kStages) {
+      if (!try_issue(n_issued == n_done)) break;
     }
     if (n_issued == n_comp) break;  // the list is exhausted (or the CTA aborted)
-    cp_async_wait_pending<kStages>(n_issued - n_comp - 1);
-    __syncwarp();  // every lane's copies of the oldest stage have landed
+    if (!wait_bar(bars + 8 * (warp * kStages + n_comp % kStages), (n_comp / kStages) & 1, vabort,
+                  status))
+      break;  // the oldest stage's K and V tiles have landed (or the CTA gave up)
 
     const int st = n_comp % kStages;
     const int pc = my_meta[2 * st], i = my_meta[2 * st + 1];
@@ -554,8 +650,9 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
 #pragma unroll
       for (int jp = 0; jp < NJ; ++jp) {
         uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
-        if (r < kMaxRows) xa = lds128(qs + (r * kChunks + 4 * jp + q4) * 16);
-        if (kRows16 && r + 8 < kMaxRows) xb = lds128(qs + ((r + 8) * kChunks + 4 * jp + q4) * 16);
+        const int cc = k_chunk(q4, jp);
+        if (r < kMaxRows) xa = lds128(qs + (r * kChunks + cc) * 16);
+        if (kRows16 && r + 8 < kMaxRows) xb = lds128(qs + ((r + 8) * kChunks + cc) * 16);
         qa[2 * jp][0] = xa.x; qa[2 * jp][1] = xa.y; qa[2 * jp + 1][0] = xa.z; qa[2 * jp + 1][1] = xa.w;
         qb[2 * jp][0] = xb.x; qb[2 * jp][1] = xb.y; qb[2 * jp + 1][0] = xb.z; qb[2 * jp + 1][1] = xb.w;
       }
@@ -573,44 +670,27 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     const int blk = inf->blk_begin + i;
     const bool blk_ok = !((bad >> st) & 1u);
     const uint32_t ks = ring + st * LY::kStageBytes;
-    const uint32_t vs = ks + LY::kTileBytes;
 
-    // ---- S = Q K^T (two 8-key halves of the block)
+    // ---- phase A: S = Q K^T (two 8-key halves of the block), each half
+    // summed in two accumulators (even and odd k-chunks) so the MMA chains
+    // are short
     float sc[2][4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      sc[h][0] = sc[h][1] = sc[h][2] = sc[h][3] = 0.f;
+      float acc2[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a) acc2[a][0] = acc2[a][1] = acc2[a][2] = acc2[a][3] = 0.f;
       const int row = 8 * h + r;
 #pragma unroll
       for (int jp = 0; jp < NJ; ++jp) {
-        const uint4 kx = lds128(ks + (row * kChunks + ((4 * jp + q4) ^ k_swz(row))) * 16);
-        mma_16816(sc[h], qa[2 * jp][0], kRows16 ? qb[2 * jp][0] : 0u, qa[2 * jp][1],
+        const uint4 kx = lds128(ks + swz128(row, k_chunk(q4, jp)));
+        mma_16816(acc2[0], qa[2 * jp][0], kRows16 ? qb[2 * jp][0] : 0u, qa[2 * jp][1],
                   kRows16 ? qb[2 * jp][1] : 0u, kx.x, kx.y);
-        mma_16816(sc[h], qa[2 * jp + 1][0], kRows16 ? qb[2 * jp + 1][0] : 0u,
+        mma_16816(acc2[1], qa[2 * jp + 1][0], kRows16 ? qb[2 * jp + 1][0] : 0u,
                   qa[2 * jp + 1][1], kRows16 ? qb[2 * jp + 1][1] : 0u, kx.z, kx.w);
       }
-    }
-    // ---- V words: keys 2q4, 2q4+1, 2q4+8, 2q4+9; 8 dims 64u+8r.. each
-    uint4 vw[4][NV];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = 2 * q4 + (e & 1) + 8 * (e >> 1);
-#pragma unroll
-      for (int u = 0; u < NV; ++u)
-        vw[e][u] = lds128(vs + (tok * kChunks + ((8 * u + r) ^ v_swz(tok))) * 16);
-    }
-    // slots of the last block past seq_len (and blocks outside the pool) may
-    // hold anything, NaN included: their V words become zeros so that the
-    // zero weights below cannot turn them into NaN in the P.V product
-    if (blk * kBlockSize + kBlockSize > L || !blk_ok) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = blk * kBlockSize + 2 * q4 + (e & 1) + 8 * (e >> 1);
-        if (!blk_ok || key >= L) {
-#pragma unroll
-          for (int u = 0; u < NV; ++u) vw[e][u] = make_uint4(0, 0, 0, 0);
-        }
-      }
+      for (int c = 0; c < 4; ++c) sc[h][c] = acc2[0][c] + acc2[1][c];
     }
     // ---- scale, mask, online softmax
     const int key0 = blk * kBlockSize + 2 * q4;  // keys key0, +1 (half 0), key0+8, +9 (half 1)
@@ -651,36 +731,52 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       l_b = l_b * al_b + (pb[0] + pb[1]) + (pb[2] + pb[3]);
       m_b = mn_b;
     }
+    ++n_comp;
+
+    // ---- phase B of the block before (same running max as O so far), then
+    // O to this block's running max
+    if (pend) phase_b();
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       o[nt][0] *= al_a; o[nt][1] *= al_a;
       if (kRows16) { o[nt][2] *= al_b; o[nt][3] *= al_b; }
     }
-    // ---- O += P V
-    const uint32_t pa0 = pack_bf16x2(pa[0], pa[1]), pa2 = pack_bf16x2(pa[2], pa[3]);
-    const uint32_t pb1 = kRows16 ? pack_bf16x2(pb[0], pb[1]) : 0u;
-    const uint32_t pb3 = kRows16 ? pack_bf16x2(pb[2], pb[3]) : 0u;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int u = nt / 8, idx = nt % 8;
-      const uint32_t sel = (idx & 1) ? 0x7632u : 0x5410u;
-      const uint32_t b0 = __byte_perm(word(vw[0][u], idx >> 1), word(vw[1][u], idx >> 1), sel);
-      const uint32_t b1 = __byte_perm(word(vw[2][u], idx >> 1), word(vw[3][u], idx >> 1), sel);
-      mma_16816(o[nt], pa0, pb1, pa2, pb3, b0, b1);
-    }
-    ++n_comp;
-    __syncwarp();  // every lane is done with this stage before it is refilled
+    pend = true;
+    pend_st = st;
+    pend_blk = blk;
+    pend_L = L;
+    pend_ok = blk_ok;
+    pp0 = pack_bf16x2(pa[0], pa[1]);
+    pp2 = pack_bf16x2(pa[2], pa[3]);
+    pp1 = kRows16 ? pack_bf16x2(pb[0], pb[1]) : 0u;
+    pp3 = kRows16 ? pack_bf16x2(pb[2], pb[3]) : 0u;
     if (i + kWarps >= inf->nb) {  // this warp's last block of the piece
+      phase_b();
+      __syncwarp();  // every lane is done with the stage before it is refilled
       if (!flush(pc, inf)) break;
     }
+    __syncwarp();  // every lane is done with the stage freed above before it is refilled
   }
-  cp_async_wait<0>();  // no copy may still target the ring when the CTA exits
+  // no TMA load may still target the ring when the CTA exits (only after a
+  // wait gave up: a normal exit has consumed every stage it loaded)
+  for (int n = n_comp; n < n_issued; ++n) {  // loaded, never waited for
+    const uint32_t b = bars + 8 * (warp * kStages + n % kStages);
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(b, (n / kStages) & 1) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
 }
 
 template <int D, int kMaxRows, bool kWriteCache>
 cudaError_t launch_one(const AttnParams& p, const DecodeWork& work, int grid,
                        cudaStream_t stream) {
   using LY = DecodeLayout<D, kMaxRows>;
+  CUtensorMap tk, tv;
+  if (!make_map(&tk, p.k_cache, D, kBlockSize, (uint64_t)p.num_blocks * p.num_kv_heads,
+                (uint64_t)D * 2, (uint64_t)kBlockSize * D * 2, kBlockSize, 1) ||
+      !make_map(&tv, p.v_cache, D, kBlockSize, (uint64_t)p.num_blocks * p.num_kv_heads,
+                (uint64_t)D * 2, (uint64_t)kBlockSize * D * 2, kBlockSize, 1))
+    return cudaErrorInvalidValue;
   auto kernel = decode_persistent_kernel<D, kMaxRows, kWriteCache>;
   static std::atomic<int> smem_done[64];
   cudaError_t e = raise_smem_limit(kernel, LY::total, smem_done);
@@ -695,7 +791,7 @@ cudaError_t launch_one(const AttnParams& p, const DecodeWork& work, int grid,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, p, work);
+  return cudaLaunchKernelEx(&cfg, kernel, p, work, tk, tv);
 }
 
 template <int D, bool kWriteCache>

@@ -56,8 +56,9 @@ constexpr int kDecodePiecesPerCta = 4;
 // needs bigger pieces to fit its partial slots
 constexpr long kDecodeMaxPieceBytes = 2l << 20;
 // pieces a launch can carry as a kernel parameter (more: the list is built on
-// the device, in the workspace); the parameter stays under 32 KB
-constexpr int kDecodeParamPieces = 1984;
+// the device, in the workspace); with the two tensor maps the launch
+// parameters stay under 32 KB
+constexpr int kDecodeParamPieces = 1920;
 
 // words of the workspace header (the first 256 bytes)
 constexpr int kWsStatus = 0;       // error bits set by a kernel that gave up waiting
