@@ -31,13 +31,19 @@
 //       the cache first when the call asks for it, and publishes the slot.
 //   compute warps 0 .. kWarps-1     warp w takes blocks w, w + kWarps, ... of
 //       every piece.  It streams them through a private ring of kStages
-//       shared-memory stages (K tile + V tile of one (block, kv-head)) with
-//       16-byte cp.async copies, up to kStages blocks in flight, and
+//       shared-memory stages (K tile + V tile of one (block, kv-head)) filled
+//       by TMA (16 x 64 boxes, one mbarrier per stage), up to kStages blocks
+//       in flight, and
 //       the ring runs on from one piece into the next without draining.  Per
-//       16-token block:
-//         S[16 rows x 16 keys] = Q . K^T     mma.m16n8k16 (two per 16 dims of D)
-//         online softmax (fp32 running max and sum, exp2 with log2(e) folded in)
-//         O[16 rows x D]      += P . V       D/8 mma.m16n8k16
+//       16-token block, with the keys on the MMA's M side and the (at most
+//       8 per n-tile) query rows on its N side, so that no MMA row is padding:
+//         S^T[16 keys x 8 rows]  = K . Q^T   mma.m16n8k16 per 16 dims of D
+//                                            (K by ldmatrix from the ring)
+//         online softmax down the columns of S^T (fp32 running max and sum,
+//         exp2 with log2(e) folded into the scale), the max moved lazily
+//         P^T: the bf16 S^T fragment transposed in registers (movmatrix)
+//         O^T[D x 8 rows]       += V^T . P^T  mma.m16n8k16 per 16 dims of D
+//                                            (V^T by ldmatrix.trans)
 //   piece merge  when a warp has computed its last block of a piece it puts
 //       its (max, sum, O) in a shared merge slot; the last warp to arrive
 //       merges them and stores the piece's result: the output rows when the
@@ -47,20 +53,18 @@
 //       warp per unit cut into several pieces merges the unit's partials
 //       into its output rows.
 //
-// The dot product's D axis is permuted identically on Q and K so that every
-// lane's B-operand words are 8 consecutive bf16 of one key row, and the
-// output's D axis is permuted so that every lane's V words are 8 consecutive
-// bf16 of one key row (undone when the output is stored).  The 16-byte chunks
-// of every tile row are XOR-swizzled on their way into shared memory so that
-// these fragment reads hit distinct banks.
+// The 16-byte chunks of every tile row are XOR-swizzled on their way into
+// shared memory (the TMA 128-byte swizzle) so that every 8 x 8 matrix that
+// ldmatrix reads hits eight distinct bank groups.
 //
 // Every wait on another warp of the CTA (a piece slot not yet published, the
 // merge slot still in use) is bounded by a time limit; one that runs out sets
 // the workspace status bit and the CTA winds down instead of hanging.  The
 // kernel is launched as a programmatic dependent of whatever precedes it on
-// the stream; it reads nothing before griddepcontrol.wait.
+// the stream; before griddepcontrol.wait it reads only its own parameters.
 #include <math.h>
 
+#include "pa_fastmath.cuh"
 #include "pa_internal.cuh"
 #include "pa_tma.cuh"
 #include "pa_wait.cuh"
@@ -69,17 +73,16 @@ namespace pa {
 namespace {
 
 // compute warps and ring stages per CTA, by head_dim and most query rows per
-// unit (shared memory: ring + merge slot + two piece slots, at most 227 KB)
-// A warp's loop over its blocks is bound by the latency of its own dependent
-// chain (loads, MMAs, shuffles, exponentials), about 2,000 cycles per block,
-// so an SM needs about a dozen compute warps to keep up with its share of
-// HBM bandwidth; the register budget of a quarter-SM (16K registers) and the
-// shared memory of the rings set how many fit.
+// unit (shared memory: ring + merge slot + two piece slots, at most 227 KB).
+// The copies a CTA keeps in flight (warps x stages x one block's K and V)
+// must cover its share of HBM bandwidth times the load latency, about 64 KB
+// to 96 KB; a warp's own loop over its blocks is bound by the latency of its
+// dependent chain (shared-memory loads, MMAs, exponentials), a few hundred
+// cycles per block.
 template <int D, int kMaxRows>
 struct DecodeCfg {
-  static constexpr int kWarps =
-      D == 64 ? (kMaxRows <= 8 ? 11 : 8) : (kMaxRows <= 4 ? 8 : kMaxRows <= 8 ? 7 : 6);
-  static constexpr int kStages = D == 64 ? 4 : 3;
+  static constexpr int kWarps = D == 64 ? 12 : (kMaxRows <= 4 ? 11 : kMaxRows <= 8 ? 10 : 8);
+  static constexpr int kStages = D == 64 ? 3 : 2;
 };
 
 // What the scheduler publishes about one piece.
@@ -100,11 +103,13 @@ struct DecodeLayout {
   static constexpr int kStageBytes = 2 * kTileBytes;     // K tile + V tile
   static constexpr int ring_off = 0;  // 1024-byte aligned (128-byte swizzle atoms)
   static constexpr int ring_bytes = kWarps * kStages * kStageBytes;
-  // merge slot: per compute warp its rows' max, sum and unnormalised O
+  // merge slot: per compute warp its rows' max, sum and unnormalised O (rows
+  // of D + 4 floats: the fragment stores of four rows hit distinct banks)
+  static constexpr int kOStride = D + 4;
   static constexpr int mm_off = ring_off + ring_bytes;                // [kWarps][kMaxRows]
   static constexpr int ml_off = mm_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows]
-  static constexpr int mo_off = ml_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows][D]
-  static constexpr int merge_end = mo_off + kWarps * kMaxRows * D * 4;
+  static constexpr int mo_off = ml_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows][kOStride]
+  static constexpr int merge_end = mo_off + kWarps * kMaxRows * kOStride * 4;
   // two piece slots: info, block ids, query rows
   static constexpr int kInfoBytes = 64;
   static constexpr int kIdsBytes = kDecodeMaxPieceBlocks * 4;
@@ -135,16 +140,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr));
   return v;
 }
 
-__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+// Four 8 x 8 bf16 matrices from shared memory (one row address per lane:
+// lanes 8i .. 8i + 7 address the rows of matrix i), as MMA fragments; the
+// .trans form delivers each matrix transposed.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&a)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&a)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+// An 8 x 8 bf16 matrix held one pair per lane (row lane / 4, columns
+// 2 (lane % 4), + 1), transposed in registers.
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
 }
 
 // CTA-scope hand-offs in shared memory: release stores, acquire loads and
@@ -167,29 +187,14 @@ __device__ __forceinline__ int add_acq_rel(int* p, int v) {
   return old;
 }
 
-// Byte offset of 16-byte chunk c of row `row` in a tile that TMA loaded as
-// 16 x 64 boxes with 128-byte swizzle: box (64-wide slice of D) c / 8 at
-// 2048 bytes per box, rows of 128 bytes, chunk c % 8 XOR row % 8.
-__device__ __forceinline__ uint32_t swz128(int row, int c) {
-  return (uint32_t)((c >> 3) * 2048 + row * 128 + (((c & 7) ^ (row & 7)) << 4));
-}
-// 16-byte chunk of a key row (and of a query row) that lane q4 holds for the
-// jp-th pair of Q.K^T MMAs: the dot product's D axis is permuted so that the
-// eight lanes of one shared-memory phase (two rows, four q4) read eight
-// distinct banks after the swizzle (rows r and r+1 differ in row % 8 bit 0).
-__device__ __forceinline__ int k_chunk(int q4, int jp) { return 8 * (jp >> 1) + 2 * q4 + (jp & 1); }
-
-// Output column c (0..7) of n-tile nt sits at dimension 64*(nt/8) + 8*c + nt%8,
-// so a lane owning columns 2*q4, 2*q4+1 of every n-tile owns, per 64-wide
-// half of D, the 16 consecutive dimensions 16*q4 .. 16*q4+15.
-__device__ __forceinline__ int out_dim(int nt, int c) { return 64 * (nt / 8) + 8 * c + (nt % 8); }
-
 // Shared control words of a CTA.
 struct DecodeCtl {
   int merged;     // CTA-local sequence number of the last piece merged (-1: none)
-  int count;      // compute warps that have put their part of the current piece in the merge slot
+  // parts of the current piece in the merge slot: the low 16 bits count the
+  // blocks they cover, bit 16 + w is set once warp w has put its part there
+  int count;
   int abort;      // set by a bounded wait that ran out: every role winds down
-  int passed[2];  // compute warps whose issue cursor has left the piece in each slot
+  int passed[2];  // compute warps with blocks in the piece in each slot whose issue cursor has left it
 };
 
 // One piece of the list (see DecodeWork): x = sequence, y = ql << 24 | rg << 22
@@ -206,11 +211,10 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   using LY = DecodeLayout<D, kMaxRows>;
   constexpr int kWarps = LY::kWarps;
   constexpr int kStages = LY::kStages;
-  constexpr bool kRows16 = kMaxRows > 8;
-  constexpr int NJ = D / 32;  // 16-byte K chunks per key row a lane reads
-  constexpr int NV = D / 64;  // 16-byte V chunks per key row a lane reads
-  constexpr int NT = D / 8;   // n-tiles of the P.V product
-  constexpr int NC = D / 16;  // k-chunks of the Q.K^T product
+  constexpr int kN = (kMaxRows + 7) / 8;  // 8-row n-tiles of query rows
+  constexpr int NK = D / 16;  // 16-dim steps of K Q^T, 16-dim m-tiles of V^T P^T
+  constexpr int kOStride = LY::kOStride;
+  constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold, log2 units
   constexpr int kChunks = D / 8;    // 16-byte chunks per tile row
   constexpr int kPanels = D / 64;   // 64-wide slices of D: one 16 x 64 TMA box each
 
@@ -252,6 +256,15 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     prefetch_tmap(&tm_v);
   }
   __syncthreads();
+  // A piece list in the kernel's parameters does not depend on the preceding
+  // kernel: its size and the CTA's first piece are read before the wait.
+  int num_pieces = 0, P = 0;
+  int4 first = make_int4(0, 0, 0, 0);
+  if (warp == kWarps && !work.from_ws) {
+    num_pieces = work.count;
+    P = work.piece_blocks;
+    if ((int)blockIdx.x < num_pieces) first = work.items[blockIdx.x];
+  }
   // Launched as a programmatic dependent: nothing the preceding kernel may
   // write is read before this wait; the next kernel may then be launched (it
   // waits for this grid in the same way).
@@ -259,19 +272,25 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   const int G = p.group;
-  const int num_pieces = work.from_ws ? p.ws_header[kWsPieceCount] : work.count;
-  const int P = work.from_ws ? p.ws_header[kWsPieceBlocks] : work.piece_blocks;
 
   if (warp == kWarps) {
     // =============================== scheduler ===============================
+    if (work.from_ws) {
+      num_pieces = p.ws_header[kWsPieceCount];
+      P = p.ws_header[kWsPieceBlocks];
+    }
+    int prev_nb = 1;  // blocks of the piece staged last
     for (int pc = 0;; ++pc) {
       // the next piece is claimed only once every block of the current one
-      // has been issued (every compute warp's issue cursor has left it; the
-      // copies then keep the warps busy for a while), so that the list's
-      // largest-first order goes to the SMs that are free
+      // has been issued (every compute warp with blocks there has moved its
+      // issue cursor past it; the copies in flight then keep the warps busy
+      // while the claim and the staging complete), so that the list's
+      // largest-first order goes to the SMs that are free.  (Claiming when
+      // the first warp moves on hides more of the staging but lets a CTA hold
+      // pieces ahead of its progress, which costs more at the list's end.)
       if (pc >= 1 &&
-          !spin_until([&] { return ld_acquire(&ctl.passed[(pc - 1) & 1]) >= kWarps; }, vabort,
-                      status))
+          !spin_until([&] { return ld_acquire(&ctl.passed[(pc - 1) & 1]) >= min(kWarps, prev_nb); },
+                      vabort, status))
         break;
       // slot pc % 2 is free once piece pc - 2 has been merged
       if (pc >= 2 &&
@@ -290,7 +309,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         }
         break;
       }
-      const int4 it = load_piece(p, work, g);
+      const int4 it = (pc == 0 && !work.from_ws) ? first : load_piece(p, work, g);
       const int s = it.x;
       const int j = it.y & 0xfff, kvh = (it.y >> 12) & 0x3ff, rg = (it.y >> 22) & 3;
       const int ql = (it.y >> 24) & 0x7f;
@@ -384,6 +403,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
           asm volatile("fence.proxy.async.global;" ::: "memory");
         }
       }
+      prev_nb = nb;
       if (lane == 0) {
         ctl.passed[pc & 1] = 0;
         inf->end = 0;
@@ -412,16 +432,32 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   const int oob_bh = p.num_blocks * p.num_kv_heads;  // first (block, kv-head) row past the pool
   const uint32_t ring = sbase + LY::ring_off + warp * kStages * LY::kStageBytes;
   int* my_meta = meta + warp * kStages * 2;
+  // ldmatrix rows this lane addresses: matrix lane / 8, row lane % 8 of it.
+  // K as the A operand (keys x dims): matrix mi holds keys 8 * (mi & 1) + 0..7
+  // of the 16-byte chunk 2 * kk + (mi >> 1); V^T as the A operand (dims x
+  // keys): matrix mi holds keys 8 * (mi >> 1) + 0..7 of chunk 2 * mt + (mi & 1).
+  // With the 128-byte swizzle, chunk c of row t sits at chunk c ^ (t % 8) of
+  // its 128-byte row, and the chunk pairs (2k, 2k + 1) never straddle a box.
+  const int mi = lane >> 3, mrow = lane & 7;
+  const uint32_t k_row = (8 * (mi & 1) + mrow) * 128;
+  const int k_hx = (mi >> 1) ^ mrow;
+  const uint32_t v_row = LY::kTileBytes + (8 * (mi >> 1) + mrow) * 128;
+  const int v_hx = (mi & 1) ^ mrow;
 
-  // the piece in slot pc, once published (nullptr before); the tag is read
-  // (with acquire order) only until the warp has seen the piece published
+  // State of piece pc's slot as this warp sees it: 0 not published yet, 1
+  // published, 2 already reused for a later piece.  The tag is read (with
+  // acquire order) only until the warp has seen the piece published.  A slot
+  // is reused for piece pc + 2 only after piece pc has been merged, which
+  // needs every warp with blocks in it: a warp that finds the slot reused had
+  // none there (it lagged behind while the piece went by) and skips it.
   int seen = -1;  // the latest piece this warp has seen published
-  auto published = [&](int pc) -> const PieceInfo* {
-    const PieceInfo* inf = slot_info(pc);
-    if (pc <= seen) return inf;
-    if (ld_acquire(&inf->tag) != pc) return nullptr;
+  auto slot_state = [&](int pc) -> int {
+    if (pc <= seen) return 1;
+    const int tag = ld_acquire(&slot_info(pc)->tag);
+    if (tag < pc) return 0;
+    if (tag > pc) return 2;
     seen = pc;
-    return inf;
+    return 1;
   };
 
   int ip = 0, ii = warp;  // issue cursor: next candidate (piece, block of the piece)
@@ -431,24 +467,32 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
 
   // Issue the copies of this warp's next block; false when there is none yet
   // (the next piece is not published and `block` is false) or none at all.
+  // Warp w takes blocks w, w + kWarps, ... of every piece: a fixed grouping,
+  // so that the piece's result does not depend on timing.
   auto try_issue = [&](bool block) -> bool {
     const PieceInfo* inf;
     while (true) {
-      inf = published(ip);
-      if (!inf) {
+      int state = slot_state(ip);
+      if (state == 0) {
         if (!block) return false;
-        if (!spin_until([&] { return published(ip) != nullptr; }, vabort, status)) {
+        if (!spin_until([&] { return (state = slot_state(ip)) != 0; }, vabort, status)) {
           issue_done = true;
           return false;
         }
-        inf = published(ip);
       }
+      if (state == 2) {  // a piece without blocks of this warp, gone by
+        ++ip;
+        ii = warp;
+        continue;
+      }
+      inf = slot_info(ip);
       if (inf->end) {
         issue_done = true;
         return false;
       }
       if (ii < inf->nb) break;
-      if (lane == 0) atomicAdd(&ctl.passed[ip & 1], 1);  // this warp leaves piece ip
+      // this warp leaves piece ip (counted when it had blocks there)
+      if (lane == 0 && warp < inf->nb) atomicAdd(&ctl.passed[ip & 1], 1);
       ++ip;
       ii = warp;
     }
@@ -472,62 +516,75 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         tma_load_3d(ks + LY::kTileBytes + pn * 2048, &tm_v, 64 * pn, 0, row_bh, bar);
       }
     }
-    if (lane == 0) {
-      my_meta[2 * st] = ip;
-      my_meta[2 * st + 1] = ii;
-    }
+    // (every lane stores the same values and reads back only what it stored)
+    my_meta[2 * st] = ip;
+    my_meta[2 * st + 1] = ii;
     ++n_issued;
     ii += kWarps;
     return true;
   };
 
-  // per-piece state of this warp
-  int cur = -1;  // piece being accumulated
-  uint32_t qa[NC][2], qb[NC][2];
-  float o[NT][4];
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-  int lim_a = 0, lim_b = 0, first_masked = 0;
+  // per-piece state of this warp.  Fragment ownership: lane (r, q4) holds the
+  // query rows 8n + 2q4 and 8n + 2q4 + 1 of n-tile n (h = 0, 1), the keys r
+  // and r + 8 of a block in S^T, and the dims 16mt + r and 16mt + r + 8 of
+  // m-tile mt in O^T.
+  int cur = -1;   // piece being accumulated
+  int n_cur = 0;  // blocks of it this warp has accumulated
+  uint32_t qf[kN][NK][2];  // Q^T as the B operand: rows 8n + r, dims 16kk + 2q4 (+8)
+  float o[kN][NK][4];      // O^T: [dim 16mt + r (+8)][row 8n + 2q4 (+1)]
+  float m[kN][2], mb[kN][2], l[kN][2];  // running max, exponent base, this lane's partial sum
+  int lim[kN][2], first_masked = 0;
 
   // The warp's part of piece pc is done: its (max, sum, O) go to the merge
   // slot; the last warp to arrive merges and stores the piece's result.
   auto flush = [&](int pc, const PieceInfo* inf) -> bool {
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-    if (kRows16) {
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-      l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-    }
+#pragma unroll
+    for (int n = 0; n < kN; ++n)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // the sum over the eight lanes holding the row's keys
+        l[n][h] += __shfl_xor_sync(0xffffffffu, l[n][h], 4);
+        l[n][h] += __shfl_xor_sync(0xffffffffu, l[n][h], 8);
+        l[n][h] += __shfl_xor_sync(0xffffffffu, l[n][h], 16);
+      }
     // the merge slot holds one piece at a time: the previous one must be merged
     if (!spin_until([&] { return ld_acquire(&ctl.merged) >= pc - 1; }, vabort, status))
       return false;
-    if (q4 == 0) {
-      if (r < kMaxRows) { msl_m[warp * kMaxRows + r] = m_a; msl_l[warp * kMaxRows + r] = l_a; }
-      if (kRows16 && r + 8 < kMaxRows) {
-        msl_m[warp * kMaxRows + r + 8] = m_b;
-        msl_l[warp * kMaxRows + r + 8] = l_b;
-      }
-    }
-    float* mo = msl_o + warp * kMaxRows * D;
+    if (r == 0) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+      for (int n = 0; n < kN; ++n)
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int d = out_dim(nt, 2 * q4 + c);
-        if (r < kMaxRows) mo[r * D + d] = o[nt][c];
-        if (kRows16 && r + 8 < kMaxRows) mo[(r + 8) * D + d] = o[nt][2 + c];
-      }
+        for (int h = 0; h < 2; ++h) {
+          const int row = 8 * n + 2 * q4 + h;
+          if (row < kMaxRows) {
+            msl_m[warp * kMaxRows + row] = m[n][h];
+            msl_l[warp * kMaxRows + row] = l[n][h];
+          }
+        }
     }
+    float* mo = msl_o + warp * kMaxRows * kOStride;
+#pragma unroll
+    for (int n = 0; n < kN; ++n)
+#pragma unroll
+      for (int mt = 0; mt < NK; ++mt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int row = 8 * n + 2 * q4 + (c & 1);
+          if (row < kMaxRows) mo[row * kOStride + 16 * mt + r + 8 * (c >> 1)] = o[n][mt][c];
+        }
     __syncwarp();
-    int last = 0;
-    if (lane == 0) last = add_acq_rel(&ctl.count, 1) + 1 == min(kWarps, inf->nb);
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) return true;
+    int parts = 0;  // once the last part is in: bit w set for every warp w with a part
+    if (lane == 0) {
+      const int add = n_cur | (1 << (16 + warp));
+      const int now = add_acq_rel(&ctl.count, add) + add;
+      parts = (now & 0xffff) == inf->nb ? now >> 16 : 0;
+    }
+    parts = __shfl_sync(0xffffffffu, parts, 0);
+    if (!parts) return true;
     __syncwarp();  // every lane reads the other warps' parts after lane 0's acquire
 
     // ---- merge the warps' parts of the piece: shared memory in, global
     // stores out, then the merge slot is free again (no round trip to global
     // memory while the other warps may wait for the slot)
-    const int nw = min(kWarps, inf->nb);
     const int rows = inf->rows, row0 = inf->row0, q0 = inf->q0;
     const int kvh = inf->kvh, rg = inf->rg, np = inf->nparts;
     const int unit = inf->s * p.num_kv_heads + kvh;
@@ -541,7 +598,8 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       // the max and the weighted sums
       float mw[kWarps];
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) mw[w] = w < nw ? msl_m[w * kMaxRows + i] : -INFINITY;
+      for (int w = 0; w < kWarps; ++w)
+        mw[w] = (parts >> w) & 1 ? msl_m[w * kMaxRows + i] : -INFINITY;
       float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mw[w]);
@@ -550,11 +608,11 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        if (w < nw) {
-          const float f = exp2f(mw[w] - base);
+        if ((parts >> w) & 1) {
+          const float f = ex2(mw[w] - base);
           Ls += msl_l[w * kMaxRows + i] * f;
-          const float4 v =
-              *reinterpret_cast<const float4*>(msl_o + (w * kMaxRows + i) * D + 4 * d4);
+          const float4 v = *reinterpret_cast<const float4*>(
+              msl_o + (w * kMaxRows + i) * kOStride + 4 * d4);
           acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
         }
       }
@@ -580,58 +638,11 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     return true;
   };
 
-  // The loop is software-pipelined by one block: iteration n computes
-  // S = Q K^T and P of block n (phase A) and adds P V of block n-1 (phase B),
-  // two independent dependency chains; O is then rescaled to block n's
-  // running max.  A block whose P.V is still pending keeps its stage.  The
-  // warp's last block of a piece finishes at once, before the piece is
-  // flushed, so nothing is pending across pieces.
-  bool pend = false;
-  int pend_st = 0, pend_blk = 0, pend_L = 0;
-  bool pend_ok = true;
-  uint32_t pp0 = 0u, pp1 = 0u, pp2 = 0u, pp3 = 0u;  // P of the pending block, bf16 pairs
-  int n_done = 0;  // blocks whose stage is free again (their P.V is in O)
-
-  auto phase_b = [&]() {  // O += P V of the pending block
-    const uint32_t vs = ring + pend_st * LY::kStageBytes + LY::kTileBytes;
-    // V words: keys 2q4, 2q4+1, 2q4+8, 2q4+9; 8 dims 64u+8r.. each
-    uint4 vw[4][NV];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = 2 * q4 + (e & 1) + 8 * (e >> 1);
-#pragma unroll
-      for (int u = 0; u < NV; ++u) vw[e][u] = lds128(vs + swz128(tok, 8 * u + r));
-    }
-    // slots of the last block past seq_len (and blocks outside the pool) may
-    // hold anything, NaN included: their V words become zeros so that the
-    // zero weights cannot turn them into NaN in the P.V product
-    if (pend_blk * kBlockSize + kBlockSize > pend_L || !pend_ok) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = pend_blk * kBlockSize + 2 * q4 + (e & 1) + 8 * (e >> 1);
-        if (!pend_ok || key >= pend_L) {
-#pragma unroll
-          for (int u = 0; u < NV; ++u) vw[e][u] = make_uint4(0, 0, 0, 0);
-        }
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int u = nt / 8, idx = nt % 8;
-      const uint32_t sel = (idx & 1) ? 0x7632u : 0x5410u;
-      const uint32_t b0 = __byte_perm(word(vw[0][u], idx >> 1), word(vw[1][u], idx >> 1), sel);
-      const uint32_t b1 = __byte_perm(word(vw[2][u], idx >> 1), word(vw[3][u], idx >> 1), sel);
-      mma_16816(o[nt], pp0, pp1, pp2, pp3, b0, b1);
-    }
-    pend = false;
-    ++n_done;
-  };
-
   while (true) {
-    // keep kStages blocks in flight (a pending block's stage included); wait
-    // for a piece to be published only when nothing is in flight
-    while (!issue_done && n_issued - n_done < kStages) {
-      if (!try_issue(n_issued == n_done)) break;
+    // keep kStages blocks in flight; wait for a piece to be published only
+    // when nothing is in flight
+    while (!issue_done && n_issued - n_comp < kStages) {
+      if (!try_issue(n_issued == n_comp)) break;
     }
     if (n_issued == n_comp) break;  // the list is exhausted (or the CTA aborted)
     if (!wait_bar(bars + 8 * (warp * kStages + n_comp % kStages), (n_comp / kStages) & 1, vabort,
@@ -643,115 +654,141 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     const PieceInfo* inf = slot_info(pc);
     const int L = inf->L;
     if (pc != cur) {
-      // ---- a new piece: its query rows as the A operand (rows r and r+8), D
-      // axis permuted as the K chunks; fresh running max, sum and O
+      // ---- a new piece: its query rows as the B operand (rows past the
+      // unit's are zero), fresh running max, sum and O
       cur = pc;
+      n_cur = 0;
       const uint32_t qs = slot_q(pc);
 #pragma unroll
-      for (int jp = 0; jp < NJ; ++jp) {
-        uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
-        const int cc = k_chunk(q4, jp);
-        if (r < kMaxRows) xa = lds128(qs + (r * kChunks + cc) * 16);
-        if (kRows16 && r + 8 < kMaxRows) xb = lds128(qs + ((r + 8) * kChunks + cc) * 16);
-        qa[2 * jp][0] = xa.x; qa[2 * jp][1] = xa.y; qa[2 * jp + 1][0] = xa.z; qa[2 * jp + 1][1] = xa.w;
-        qb[2 * jp][0] = xb.x; qb[2 * jp][1] = xb.y; qb[2 * jp + 1][0] = xb.z; qb[2 * jp + 1][1] = xb.w;
-      }
+      for (int n = 0; n < kN; ++n) {
+        const int row = 8 * n + r;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-      m_a = m_b = -INFINITY;
-      l_a = l_b = 0.f;
+        for (int kk = 0; kk < NK; ++kk) {
+          qf[n][kk][0] = row < kMaxRows ? lds32(qs + (row * D + 16 * kk + 2 * q4) * 2) : 0u;
+          qf[n][kk][1] = row < kMaxRows ? lds32(qs + (row * D + 16 * kk + 8 + 2 * q4) * 2) : 0u;
+        }
+      }
       const int rows = inf->rows, ql = inf->ql;
-      // causal limit of rows r and r+8: query j sees keys <= L - ql + j
-      lim_a = L - ql + (inf->row0 + min(r, rows - 1)) / G;
-      lim_b = L - ql + (inf->row0 + min(r + 8, rows - 1)) / G;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) {
+#pragma unroll
+        for (int mt = 0; mt < NK; ++mt) o[n][mt][0] = o[n][mt][1] = o[n][mt][2] = o[n][mt][3] = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          m[n][h] = -INFINITY;
+          mb[n][h] = 0.f;
+          l[n][h] = 0.f;
+          // causal limit of the row: query j of the sequence sees keys <= L - ql + j
+          lim[n][h] = L - ql + (inf->row0 + min(8 * n + 2 * q4 + h, rows - 1)) / G;
+        }
+      }
       first_masked = L - ql + 1;  // keys at or beyond this may be masked for some row
     }
 
-    const int blk = inf->blk_begin + i;
+    const int kb = (inf->blk_begin + i) * kBlockSize;  // first key of the block
     const bool blk_ok = !((bad >> st) & 1u);
     const uint32_t ks = ring + st * LY::kStageBytes;
 
-    // ---- phase A: S = Q K^T (two 8-key halves of the block), each half
-    // summed in two accumulators (even and odd k-chunks) so the MMA chains
-    // are short
-    float sc[2][4];
+    // ---- S^T = K Q^T: keys on the MMA's M side, query rows on N; per n-tile
+    // two accumulators (even and odd 16-dim steps) keep the chains short
+    float x[kN][4];
+    {
+      float sa[kN][2][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float acc2[2][4];
+      for (int n = 0; n < kN; ++n)
 #pragma unroll
-      for (int a = 0; a < 2; ++a) acc2[a][0] = acc2[a][1] = acc2[a][2] = acc2[a][3] = 0.f;
-      const int row = 8 * h + r;
+        for (int a = 0; a < 2; ++a) sa[n][a][0] = sa[n][a][1] = sa[n][a][2] = sa[n][a][3] = 0.f;
 #pragma unroll
-      for (int jp = 0; jp < NJ; ++jp) {
-        const uint4 kx = lds128(ks + swz128(row, k_chunk(q4, jp)));
-        mma_16816(acc2[0], qa[2 * jp][0], kRows16 ? qb[2 * jp][0] : 0u, qa[2 * jp][1],
-                  kRows16 ? qb[2 * jp][1] : 0u, kx.x, kx.y);
-        mma_16816(acc2[1], qa[2 * jp + 1][0], kRows16 ? qb[2 * jp + 1][0] : 0u,
-                  qa[2 * jp + 1][1], kRows16 ? qb[2 * jp + 1][1] : 0u, kx.z, kx.w);
+      for (int kk = 0; kk < NK; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(a, ks + (kk >> 2) * 2048 + k_row + ((((2 * kk) & 7) ^ k_hx) << 4));
+#pragma unroll
+        for (int n = 0; n < kN; ++n)
+          mma_16816(sa[n][kk & 1], a[0], a[1], a[2], a[3], qf[n][kk][0], qf[n][kk][1]);
       }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) sc[h][c] = acc2[0][c] + acc2[1][c];
-    }
-    // ---- scale, mask, online softmax
-    const int key0 = blk * kBlockSize + 2 * q4;  // keys key0, +1 (half 0), key0+8, +9 (half 1)
-    const bool tail = (blk * kBlockSize + kBlockSize > first_masked) || !blk_ok;
-    float xa[4], xb[4];
+      for (int n = 0; n < kN; ++n)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int key = key0 + (e & 1) + 8 * (e >> 1);
-      xa[e] = sc[e >> 1][e & 1] * p.scale_log2;
-      xb[e] = sc[e >> 1][2 + (e & 1)] * p.scale_log2;
-      if (tail) {
-        if (!blk_ok || key > lim_a) xa[e] = -INFINITY;
-        if (!blk_ok || key > lim_b) xb[e] = -INFINITY;
+        for (int c = 0; c < 4; ++c) x[n][c] = (sa[n][0][c] + sa[n][1][c]) * p.scale_log2;
+    }
+    // ---- mask: keys past a row's causal limit (past seq_len for a decode)
+    // and every key of a block outside the pool
+    if (kb + kBlockSize > first_masked || !blk_ok) {
+#pragma unroll
+      for (int n = 0; n < kN; ++n)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (!blk_ok || kb + r + 8 * (c >> 1) > lim[n][c & 1]) x[n][c] = -INFINITY;
+    }
+    // ---- online softmax with a lazy rescale: the running max of a row moves
+    // (and O and the sums are rescaled) only when some score exceeds it by
+    // more than kRescaleLog2, so exp2(score - base) stays below
+    // 2^kRescaleLog2 and most blocks skip the row reduction
+    bool need = false;
+#pragma unroll
+    for (int n = 0; n < kN; ++n)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) need |= fmaxf(x[n][h], x[n][h + 2]) > m[n][h] + kRescaleLog2;
+    if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+      for (int n = 0; n < kN; ++n)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float bm = fmaxf(x[n][h], x[n][h + 2]);
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+          const float mn = fmaxf(m[n][h], bm);
+          if (mn > m[n][h]) {
+            const float al = ex2(m[n][h] - mn);  // 0 while the row had no finite score
+            m[n][h] = mn;
+            mb[n][h] = mn;
+            l[n][h] *= al;
+#pragma unroll
+            for (int mt = 0; mt < NK; ++mt) {
+              o[n][mt][h] *= al;
+              o[n][mt][h + 2] *= al;
+            }
+          }
+        }
+    }
+    // ---- P^T as the B operand of O^T += V^T P^T: the bf16 pairs of P in the
+    // S^T fragment (keys r / r + 8, rows 2q4, 2q4 + 1) are transposed 8 x 8 to
+    // the B fragment (keys 2q4, 2q4 + 1 / + 8, row r)
+    uint32_t pb[kN][2];
+#pragma unroll
+    for (int n = 0; n < kN; ++n) {
+      float pr[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) pr[c] = ex2(x[n][c] - mb[n][c & 1]);
+      l[n][0] += pr[0] + pr[2];
+      l[n][1] += pr[1] + pr[3];
+      pb[n][0] = movm_t(pack_bf16x2(pr[0], pr[1]));
+      pb[n][1] = movm_t(pack_bf16x2(pr[2], pr[3]));
+    }
+    // slots of the last block past seq_len (and blocks outside the pool) may
+    // hold anything, NaN included: their V elements become zeros so that the
+    // zero weights cannot turn them into NaN in the P.V product
+    uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;  // keys 2q4, 2q4 + 1 / 2q4 + 8, 2q4 + 9
+    const bool vtail = kb + kBlockSize > L || !blk_ok;
+    if (vtail) {
+      const int k0 = kb + 2 * q4;
+      vm0 = !blk_ok ? 0u : (k0 < L ? 0xffffu : 0u) | (k0 + 1 < L ? 0xffff0000u : 0u);
+      vm1 = !blk_ok ? 0u : (k0 + 8 < L ? 0xffffu : 0u) | (k0 + 9 < L ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int mt = 0; mt < NK; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_t(a, ks + (mt >> 2) * 2048 + v_row + ((((2 * mt) & 7) ^ v_hx) << 4));
+      if (vtail) {
+        a[0] &= vm0; a[1] &= vm0; a[2] &= vm1; a[3] &= vm1;
       }
-    }
-    float bm_a = fmaxf(fmaxf(xa[0], xa[1]), fmaxf(xa[2], xa[3]));
-    bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 1));
-    bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 2));
-    const float mn_a = fmaxf(m_a, bm_a);
-    const float base_a = (mn_a == -INFINITY) ? 0.f : mn_a;
-    const float al_a = exp2f(m_a - base_a);
-    float pa[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) pa[e] = exp2f(xa[e] - base_a);
-    l_a = l_a * al_a + (pa[0] + pa[1]) + (pa[2] + pa[3]);
-    m_a = mn_a;
-    float pb[4] = {0.f, 0.f, 0.f, 0.f};
-    float al_b = 1.f;
-    if (kRows16) {
-      float bm_b = fmaxf(fmaxf(xb[0], xb[1]), fmaxf(xb[2], xb[3]));
-      bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 1));
-      bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 2));
-      const float mn_b = fmaxf(m_b, bm_b);
-      const float base_b = (mn_b == -INFINITY) ? 0.f : mn_b;
-      al_b = exp2f(m_b - base_b);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) pb[e] = exp2f(xb[e] - base_b);
-      l_b = l_b * al_b + (pb[0] + pb[1]) + (pb[2] + pb[3]);
-      m_b = mn_b;
+      for (int n = 0; n < kN; ++n) mma_16816(o[n][mt], a[0], a[1], a[2], a[3], pb[n][0], pb[n][1]);
     }
     ++n_comp;
-
-    // ---- phase B of the block before (same running max as O so far), then
-    // O to this block's running max
-    if (pend) phase_b();
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      o[nt][0] *= al_a; o[nt][1] *= al_a;
-      if (kRows16) { o[nt][2] *= al_b; o[nt][3] *= al_b; }
-    }
-    pend = true;
-    pend_st = st;
-    pend_blk = blk;
-    pend_L = L;
-    pend_ok = blk_ok;
-    pp0 = pack_bf16x2(pa[0], pa[1]);
-    pp2 = pack_bf16x2(pa[2], pa[3]);
-    pp1 = kRows16 ? pack_bf16x2(pb[0], pb[1]) : 0u;
-    pp3 = kRows16 ? pack_bf16x2(pb[2], pb[3]) : 0u;
+    ++n_cur;
     if (i + kWarps >= inf->nb) {  // this warp's last block of the piece
-      phase_b();
       __syncwarp();  // every lane is done with the stage before it is refilled
       if (!flush(pc, inf)) break;
     }
@@ -1026,7 +1063,7 @@ decode_combine_kernel(const AttnParams p, int piece_blocks, int from_ws) {
     for (int q = 0; q < np; ++q) {
       const int64_t sl = uslot + q * step + i;
       const float2 ml = __ldcg(pml + sl);
-      const float f = exp2f(ml.x - base);
+      const float f = ex2(ml.x - base);
       const float4 v = __ldcg(po + sl * D4 + d4);
       Ls += ml.y * f;
       acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
