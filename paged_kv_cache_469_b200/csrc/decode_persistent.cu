@@ -64,6 +64,13 @@
 // the stream; before griddepcontrol.wait it reads only its own parameters.
 #include <math.h>
 
+#include <algorithm>
+#include <cstring>
+#include <functional>
+#include <queue>
+#include <utility>
+#include <vector>
+
 #include "pa_fastmath.cuh"
 #include "pa_internal.cuh"
 #include "pa_tma.cuh"
@@ -93,6 +100,7 @@ struct PieceInfo {
   int blk_begin, nb;  // the piece's blocks: blk_begin .. blk_begin + nb - 1 of the sequence
   int L, ql, q0;
   int rows, row0;  // this unit's query rows: global rows row0 .. row0 + rows - 1
+  int rot;         // block subset c of the piece (blocks c, c + kWarps, ...) goes to warp (c + rot) % kWarps
 };
 
 template <int D, int kMaxRows>
@@ -109,7 +117,9 @@ struct DecodeLayout {
   static constexpr int mm_off = ring_off + ring_bytes;                // [kWarps][kMaxRows]
   static constexpr int ml_off = mm_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows]
   static constexpr int mo_off = ml_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows][kOStride]
-  static constexpr int merge_end = mo_off + kWarps * kMaxRows * kOStride * 4;
+  // the merged rows' max and sum
+  static constexpr int rs_off = mo_off + kWarps * kMaxRows * kOStride * 4;  // [2][kMaxRows]
+  static constexpr int merge_end = rs_off + 2 * kMaxRows * 4;
   // two piece slots: info, block ids, query rows
   static constexpr int kInfoBytes = 64;
   static constexpr int kIdsBytes = kDecodeMaxPieceBlocks * 4;
@@ -238,6 +248,8 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   float* msl_m = reinterpret_cast<float*>(smem + LY::mm_off);
   float* msl_l = reinterpret_cast<float*>(smem + LY::ml_off);
   float* msl_o = reinterpret_cast<float*>(smem + LY::mo_off);
+  float* row_m = reinterpret_cast<float*>(smem + LY::rs_off);
+  float* row_l = row_m + kMaxRows;
   int* meta = reinterpret_cast<int*>(smem + LY::meta_off);  // [kWarps][kStages][2]
   const uint32_t bars = sbase + LY::bar_off;                 // [kWarps][kStages] mbarriers
   volatile int* vabort = &ctl.abort;
@@ -258,12 +270,19 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   __syncthreads();
   // A piece list in the kernel's parameters does not depend on the preceding
   // kernel: its size and the CTA's first piece are read before the wait.
-  int num_pieces = 0, P = 0;
+  int num_pieces = 0, P = 0, g_begin = 0, g_end = 0;
   int4 first = make_int4(0, 0, 0, 0);
   if (warp == kWarps && !work.from_ws) {
     num_pieces = work.count;
     P = work.piece_blocks;
-    if ((int)blockIdx.x < num_pieces) first = work.items[blockIdx.x];
+    if (work.dealt) {
+      g_begin = work.cta_off[blockIdx.x];
+      g_end = work.cta_off[blockIdx.x + 1];
+    } else {
+      g_begin = blockIdx.x;
+      g_end = num_pieces;
+    }
+    if (g_begin < g_end) first = work.items[g_begin];
   }
   // Launched as a programmatic dependent: nothing the preceding kernel may
   // write is read before this wait; the next kernel may then be launched (it
@@ -278,8 +297,15 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     if (work.from_ws) {
       num_pieces = p.ws_header[kWsPieceCount];
       P = p.ws_header[kWsPieceBlocks];
+      g_begin = blockIdx.x;
+      g_end = num_pieces;
     }
+    const bool dealt = !work.from_ws && work.dealt;
     int prev_nb = 1;  // blocks of the piece staged last
+    // the CTA's pieces are dealt to the compute warps as one round-robin:
+    // each piece starts at the warp after the one that got the previous
+    // piece's last block, so that no warp gets every piece's ragged remainder
+    int rot = 0;
     for (int pc = 0;; ++pc) {
       // the next piece is claimed only once every block of the current one
       // has been issued (every compute warp with blocks there has moved its
@@ -288,7 +314,8 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       // largest-first order goes to the SMs that are free.  (Claiming when
       // the first warp moves on hides more of the staging but lets a CTA hold
       // pieces ahead of its progress, which costs more at the list's end.)
-      if (pc >= 1 &&
+      // (pieces dealt on the host are staged as soon as their slot is free)
+      if (pc >= 1 && !dealt &&
           !spin_until([&] { return ld_acquire(&ctl.passed[(pc - 1) & 1]) >= min(kWarps, prev_nb); },
                       vabort, status))
         break;
@@ -296,13 +323,13 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       if (pc >= 2 &&
           !spin_until([&] { return ld_acquire(&ctl.merged) >= pc - 2; }, vabort, status))
         break;
-      int g = blockIdx.x;
-      if (pc > 0) {
+      int g = g_begin + pc;
+      if (pc > 0 && !dealt) {
         if (lane == 0) g = gridDim.x + atomicAdd(p.ws_header + kWsClaim, 1);
         g = __shfl_sync(0xffffffffu, g, 0);
       }
       PieceInfo* inf = slot_info(pc);
-      if (g >= num_pieces) {
+      if (g >= g_end) {
         if (lane == 0) {
           inf->end = 1;
           st_release(&inf->tag, pc);
@@ -411,12 +438,14 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         inf->blk_begin = blk_begin; inf->nb = nb;
         inf->L = L; inf->ql = ql; inf->q0 = q0;
         inf->rows = rows; inf->row0 = row0;
+        inf->rot = rot;
       }
+      rot = (rot + nb) % kWarps;
       __syncwarp();
       if (lane == 0) st_release(&inf->tag, pc);
     }
     // the last CTA to finish claiming resets the claim counter for the next call
-    if (lane == 0) {
+    if (lane == 0 && !dealt) {
       __threadfence();
       const int prev = atomicAdd(p.ws_header + kWsDone, 1);
       if (prev == (int)gridDim.x - 1) {
@@ -460,15 +489,16 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     return 1;
   };
 
-  int ip = 0, ii = warp;  // issue cursor: next candidate (piece, block of the piece)
+  int ip = 0, ii = -1;  // issue cursor: next candidate (piece, block of the piece; -1: its first)
   bool issue_done = false;
   int n_issued = 0, n_comp = 0;
   uint32_t bad = 0;  // bit (stage): that stage's block id was outside the pool
 
   // Issue the copies of this warp's next block; false when there is none yet
   // (the next piece is not published and `block` is false) or none at all.
-  // Warp w takes blocks w, w + kWarps, ... of every piece: a fixed grouping,
-  // so that the piece's result does not depend on timing.
+  // Warp w takes the blocks c, c + kWarps, ... of every piece, c = (w - rot)
+  // mod kWarps: a fixed grouping, so that the piece's result does not depend
+  // on timing.
   auto try_issue = [&](bool block) -> bool {
     const PieceInfo* inf;
     while (true) {
@@ -482,7 +512,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       }
       if (state == 2) {  // a piece without blocks of this warp, gone by
         ++ip;
-        ii = warp;
+        ii = -1;
         continue;
       }
       inf = slot_info(ip);
@@ -490,11 +520,13 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         issue_done = true;
         return false;
       }
+      const int first = (warp - inf->rot + kWarps) % kWarps;
+      if (ii < 0) ii = first;
       if (ii < inf->nb) break;
       // this warp leaves piece ip (counted when it had blocks there)
-      if (lane == 0 && warp < inf->nb) atomicAdd(&ctl.passed[ip & 1], 1);
+      if (lane == 0 && first < inf->nb) atomicAdd(&ctl.passed[ip & 1], 1);
       ++ip;
-      ii = warp;
+      ii = -1;
     }
     const int st = n_issued % kStages;
     const int id = slot_ids(ip)[ii];
@@ -584,49 +616,88 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
 
     // ---- merge the warps' parts of the piece: shared memory in, global
     // stores out, then the merge slot is free again (no round trip to global
-    // memory while the other warps may wait for the slot)
+    // memory while the other warps may wait for the slot).  The parts are
+    // combined in block-subset order whichever warp merges, so the result
+    // does not depend on timing or on the piece's rotation.
     const int rows = inf->rows, row0 = inf->row0, q0 = inf->q0;
-    const int kvh = inf->kvh, rg = inf->rg, np = inf->nparts;
+    const int kvh = inf->kvh, rg = inf->rg, np = inf->nparts, rot = inf->rot;
     const int unit = inf->s * p.num_kv_heads + kvh;
     __nv_bfloat16* out = (__nv_bfloat16*)p.out;
     constexpr int D4 = D / 4;
     const bool direct = np == 1;
     const int64_t slot0 = ((int64_t)unit * p.max_parts + inf->j * p.row_groups + rg) * kDecodeRows;
-    for (int e = lane; e < rows * D4; e += 32) {
-      const int i = e / D4, d4 = e % D4;
-      // every warp's value loaded first (unrolled over the CTA's warps), then
-      // the max and the weighted sums
-      float mw[kWarps];
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w)
-        mw[w] = (parts >> w) & 1 ? msl_m[w * kMaxRows + i] : -INFINITY;
+    {
+      // per row: the max over the parts, each part's weight 2^(m_w - max)
+      // (written over its max), and the weighted sum of the parts' sums; the
+      // 32 / kMaxRows lanes of a row share its parts, taken in block-subset
+      // order (subset c: warp (c + rot) % kWarps)
+      constexpr int W = 32 / kMaxRows;
+      constexpr int kPer = (kWarps + W - 1) / W;
+      const int i = lane % kMaxRows, wg = lane / kMaxRows;
+      float mv[kPer], lv[kPer];
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mw[w]);
+      for (int k = 0; k < kPer; ++k) {
+        const int c = wg + W * k, w = (c + rot) % kWarps;
+        const bool has = c < kWarps && ((parts >> w) & 1);
+        mv[k] = has ? msl_m[w * kMaxRows + i] : -INFINITY;
+        lv[k] = has ? msl_l[w * kMaxRows + i] : 0.f;
+        M = fmaxf(M, mv[k]);
+      }
+#pragma unroll
+      for (int off = kMaxRows; off < 32; off <<= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
       const float base = (M == -INFINITY) ? 0.f : M;
       float Ls = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        if ((parts >> w) & 1) {
-          const float f = ex2(mw[w] - base);
-          Ls += msl_l[w * kMaxRows + i] * f;
-          const float4 v = *reinterpret_cast<const float4*>(
-              msl_o + (w * kMaxRows + i) * kOStride + 4 * d4);
-          acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
-        }
+      for (int k = 0; k < kPer; ++k) {
+        const int c = wg + W * k, w = (c + rot) % kWarps;
+        const float wt = ex2(mv[k] - base);  // 0 for a missing part
+        Ls += lv[k] * wt;
+        if (c < kWarps) msl_m[w * kMaxRows + i] = wt;
       }
+#pragma unroll
+      for (int off = kMaxRows; off < 32; off <<= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+      if (wg == 0) {
+        row_m[i] = M;
+        row_l[i] = Ls;
+      }
+    }
+    __syncwarp();
+    // the weighted sums of the parts' O rows, then the stores; the merge slot
+    // is released last.  The parts present are block subsets 0 .. nw - 1 (a
+    // subset has blocks when c < nb).  This code runs once per piece, so it is
+    // kept compact: cold in the instruction cache, an unrolled form costs more
+    // in fetches than its loads.
+    const int nw = min(kWarps, inf->nb);
+    for (int e = lane; e < rows * D4; e += 32) {
+      const int i = e / D4, d4 = e % D4;
+      const float* wrow = msl_m + i;
+      const float* orow = msl_o + i * kOStride + 4 * d4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      int w = rot;
+#pragma unroll 4
+      for (int c = 0; c < nw; ++c) {
+        const float wt = wrow[w * kMaxRows];
+        const float4 v = *reinterpret_cast<const float4*>(orow + w * (kMaxRows * kOStride));
+        acc.x = fmaf(v.x, wt, acc.x);
+        acc.y = fmaf(v.y, wt, acc.y);
+        acc.z = fmaf(v.z, wt, acc.z);
+        acc.w = fmaf(v.w, wt, acc.w);
+        w = w + 1 == kWarps ? 0 : w + 1;
+      }
+      const float Ls = row_l[i];
       if (direct) {
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
         const int gi = row0 + i;
         const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
         uint2 pk;
         pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
         pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
         *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
       } else {
         reinterpret_cast<float4*>(p.ws_o)[(slot0 + i) * D4 + d4] = acc;
-        if (d4 == 0) reinterpret_cast<float2*>(p.ws_ml)[slot0 + i] = make_float2(M, Ls);
+        if (d4 == 0) reinterpret_cast<float2*>(p.ws_ml)[slot0 + i] = make_float2(row_m[i], Ls);
       }
     }
     __syncwarp();  // every lane is done with the merge slot and the piece slot
@@ -1014,7 +1085,48 @@ bool host_piece_list(DecodeWork* work, const AttnParams& p, const int32_t* seq_l
   work->piece_blocks = P;
   work->from_ws = 0;
   work->split = mx > P;  // some unit has more than one piece
+  work->dealt = 0;
   return true;
+}
+
+// Deals the list's pieces (longest first) to `ctas` CTAs: each to the CTA
+// with the least work so far, a piece costing its blocks plus
+// kDecodePieceCostBlocks.  CTA b's pieces then sit at items cta_off[b] ..
+// cta_off[b + 1] - 1, in the order dealt, so that each CTA can stage its next
+// piece while the current one streams instead of claiming it when it is
+// nearly done.  (The claims of a shared counter adapt to SMs that run slower,
+// but every claim's round trips and staging then sit on the CTA's path.)
+constexpr int kDecodeDealPiecesPerCta = 4;
+
+void deal_pieces(DecodeWork* work, int ctas) {
+  const int n = work->count, P = work->piece_blocks;
+  if (ctas <= 0 || ctas > kDecodeMaxDealtCtas || n < ctas) return;
+  static thread_local int4 items[kDecodeParamPieces];
+  static thread_local int owner[kDecodeParamPieces];
+  static thread_local int count[kDecodeMaxDealtCtas];
+  using Load = std::pair<long long, int>;  // (work so far, CTA)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int b = 0; b < ctas; ++b) {
+    heap.push({0, b});
+    count[b] = 0;
+  }
+  for (int g = 0; g < n; ++g) {  // the list is longest first
+    const int4 it = work->items[g];
+    const int nblk = (it.z + kBlockSize - 1) / kBlockSize, j = it.y & 0xfff;
+    const int nb = std::min(P, nblk - j * P);
+    Load l = heap.top();
+    heap.pop();
+    owner[g] = l.second;
+    ++count[l.second];
+    l.first += nb + kDecodePieceCostBlocks;
+    heap.push(l);
+  }
+  work->cta_off[0] = 0;
+  for (int b = 0; b < ctas; ++b) work->cta_off[b + 1] = work->cta_off[b] + count[b];
+  for (int b = 0; b < ctas; ++b) count[b] = work->cta_off[b];
+  for (int g = 0; g < n; ++g) items[count[owner[g]]++] = work->items[g];
+  std::memcpy(work->items, items, sizeof(int4) * n);
+  work->dealt = 1;
 }
 
 // ------------------------------------------------------------------ combine
@@ -1114,18 +1226,25 @@ cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_
                           int max_ctas_allowed) {
   if (p.num_seqs == 0) return cudaSuccess;
   const int max_rows = max(1, min(p.decode_rows, kDecodeRows));  // rows of one unit at most
-  const int ctas = max(1, min(max_ctas(head_dim, max_rows), max_ctas_allowed));
-  static thread_local DecodeWork work;  // 16 KB: kept off the stack
+  const int full = max_ctas(head_dim, max_rows);
+  const int ctas = max(1, min(full, max_ctas_allowed));
+  static thread_local DecodeWork work;  // 30 KB: kept off the stack
   int grid = ctas;
   if (seq_lens_host && query_start_loc_host &&
       host_piece_list(&work, p, seq_lens_host, query_start_loc_host, ctas, head_dim)) {
     if (work.count == 0) return cudaSuccess;
     grid = min(ctas, work.count);
+    // Dealt on the host when the kernel has every SM to itself and each CTA
+    // gets several pieces: the claims' latency then adds up on every CTA.
+    // With few pieces per CTA, or SMs shared with a prefill running beside
+    // it, the claims' adapting to each SM's actual pace is worth more.
+    if (ctas == full && work.count >= kDecodeDealPiecesPerCta * grid) deal_pieces(&work, grid);
   } else {
     work.count = 0;
     work.piece_blocks = 0;
     work.from_ws = 1;
     work.split = 1;
+    work.dealt = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(1024);

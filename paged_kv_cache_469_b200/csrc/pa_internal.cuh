@@ -56,9 +56,14 @@ constexpr int kDecodePiecesPerCta = 4;
 // needs bigger pieces to fit its partial slots
 constexpr long kDecodeMaxPieceBytes = 2l << 20;
 // pieces a launch can carry as a kernel parameter (more: the list is built on
-// the device, in the workspace); with the two tensor maps the launch
-// parameters stay under 32 KB
-constexpr int kDecodeParamPieces = 1920;
+// the device, in the workspace); with the per-CTA offsets and the two tensor
+// maps the launch parameters stay under 32 KB
+constexpr int kDecodeParamPieces = 1792;
+// a list in the kernel parameters is dealt to at most this many CTAs on the
+// host (longest first, each to the CTA with the least work so far, a piece
+// counted as its blocks plus kDecodePieceCostBlocks for its staging and merge)
+constexpr int kDecodeMaxDealtCtas = 256;
+constexpr int kDecodePieceCostBlocks = 8;
 
 // words of the workspace header (the first 256 bytes)
 constexpr int kWsStatus = 0;       // error bits set by a kernel that gave up waiting
@@ -117,6 +122,8 @@ struct DecodeWork {
   int piece_blocks;
   int from_ws;
   int split;  // some unit has more than one piece (its partials need the combine kernel)
+  int dealt;  // CTA b takes items cta_off[b] .. cta_off[b + 1] - 1 (else: claims from a counter)
+  int cta_off[kDecodeMaxDealtCtas + 1];
   int4 items[kDecodeParamPieces];
 };
 
