@@ -68,6 +68,7 @@
 #include <cstring>
 #include <functional>
 #include <queue>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -156,6 +157,14 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 // Four 8 x 8 bf16 matrices from shared memory (one row address per lane:
 // lanes 8i .. 8i + 7 address the rows of matrix i), as MMA fragments; the
 // .trans form delivers each matrix transposed.
@@ -200,9 +209,7 @@ __device__ __forceinline__ int add_acq_rel(int* p, int v) {
 // Shared control words of a CTA.
 struct DecodeCtl {
   int merged;     // CTA-local sequence number of the last piece merged (-1: none)
-  // parts of the current piece in the merge slot: the low 16 bits count the
-  // blocks they cover, bit 16 + w is set once warp w has put its part there
-  int count;
+  int count;      // blocks covered by the parts of the current piece in the merge slot
   int abort;      // set by a bounded wait that ran out: every role winds down
   int passed[2];  // compute warps with blocks in the piece in each slot whose issue cursor has left it
 };
@@ -578,9 +585,12 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         l[n][h] += __shfl_xor_sync(0xffffffffu, l[n][h], 8);
         l[n][h] += __shfl_xor_sync(0xffffffffu, l[n][h], 16);
       }
-    // the merge slot holds one piece at a time: the previous one must be merged
+    // the merge slot holds one piece at a time: the previous one must be
+    // merged.  The warp's part goes to the place of its block subset c.
     if (!spin_until([&] { return ld_acquire(&ctl.merged) >= pc - 1; }, vabort, status))
       return false;
+    const int rot = inf->rot;
+    const int sub = warp >= rot ? warp - rot : warp - rot + kWarps;
     if (r == 0) {
 #pragma unroll
       for (int n = 0; n < kN; ++n)
@@ -588,12 +598,12 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         for (int h = 0; h < 2; ++h) {
           const int row = 8 * n + 2 * q4 + h;
           if (row < kMaxRows) {
-            msl_m[warp * kMaxRows + row] = m[n][h];
-            msl_l[warp * kMaxRows + row] = l[n][h];
+            msl_m[sub * kMaxRows + row] = m[n][h];
+            msl_l[sub * kMaxRows + row] = l[n][h];
           }
         }
     }
-    float* mo = msl_o + warp * kMaxRows * kOStride;
+    float* mo = msl_o + sub * kMaxRows * kOStride;
 #pragma unroll
     for (int n = 0; n < kN; ++n)
 #pragma unroll
@@ -604,33 +614,29 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
           if (row < kMaxRows) mo[row * kOStride + 16 * mt + r + 8 * (c >> 1)] = o[n][mt][c];
         }
     __syncwarp();
-    int parts = 0;  // once the last part is in: bit w set for every warp w with a part
-    if (lane == 0) {
-      const int add = n_cur | (1 << (16 + warp));
-      const int now = add_acq_rel(&ctl.count, add) + add;
-      parts = (now & 0xffff) == inf->nb ? now >> 16 : 0;
-    }
-    parts = __shfl_sync(0xffffffffu, parts, 0);
-    if (!parts) return true;
+    int last = 0;  // the blocks of every part are in: this warp merges
+    if (lane == 0) last = add_acq_rel(&ctl.count, n_cur) + n_cur == inf->nb;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return true;
     __syncwarp();  // every lane reads the other warps' parts after lane 0's acquire
 
     // ---- merge the warps' parts of the piece: shared memory in, global
     // stores out, then the merge slot is free again (no round trip to global
     // memory while the other warps may wait for the slot).  The parts are
-    // combined in block-subset order whichever warp merges, so the result
-    // does not depend on timing or on the piece's rotation.
+    // placed and combined in block-subset order whichever warp merges, so the
+    // result does not depend on timing or on the piece's rotation.
     const int rows = inf->rows, row0 = inf->row0, q0 = inf->q0;
-    const int kvh = inf->kvh, rg = inf->rg, np = inf->nparts, rot = inf->rot;
+    const int kvh = inf->kvh, rg = inf->rg, np = inf->nparts, ql = inf->ql;
+    const int nw = min(kWarps, inf->nb);  // parts present: block subsets 0 .. nw - 1
     const int unit = inf->s * p.num_kv_heads + kvh;
     __nv_bfloat16* out = (__nv_bfloat16*)p.out;
     constexpr int D4 = D / 4;
     const bool direct = np == 1;
     const int64_t slot0 = ((int64_t)unit * p.max_parts + inf->j * p.row_groups + rg) * kDecodeRows;
     {
-      // per row: the max over the parts, each part's weight 2^(m_w - max)
+      // per row: the max over the parts, each part's weight 2^(m_c - max)
       // (written over its max), and the weighted sum of the parts' sums; the
-      // 32 / kMaxRows lanes of a row share its parts, taken in block-subset
-      // order (subset c: warp (c + rot) % kWarps)
+      // 32 / kMaxRows lanes of a row share its parts
       constexpr int W = 32 / kMaxRows;
       constexpr int kPer = (kWarps + W - 1) / W;
       const int i = lane % kMaxRows, wg = lane / kMaxRows;
@@ -638,10 +644,10 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       float M = -INFINITY;
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
-        const int c = wg + W * k, w = (c + rot) % kWarps;
-        const bool has = c < kWarps && ((parts >> w) & 1);
-        mv[k] = has ? msl_m[w * kMaxRows + i] : -INFINITY;
-        lv[k] = has ? msl_l[w * kMaxRows + i] : 0.f;
+        const int c = wg + W * k;
+        const bool has = c < nw;
+        mv[k] = has ? msl_m[c * kMaxRows + i] : -INFINITY;
+        lv[k] = has ? msl_l[c * kMaxRows + i] : 0.f;
         M = fmaxf(M, mv[k]);
       }
 #pragma unroll
@@ -651,10 +657,10 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       float Ls = 0.f;
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
-        const int c = wg + W * k, w = (c + rot) % kWarps;
+        const int c = wg + W * k;
         const float wt = ex2(mv[k] - base);  // 0 for a missing part
         Ls += lv[k] * wt;
-        if (c < kWarps) msl_m[w * kMaxRows + i] = wt;
+        if (c < kWarps) msl_m[c * kMaxRows + i] = wt;
       }
 #pragma unroll
       for (int off = kMaxRows; off < 32; off <<= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
@@ -664,33 +670,56 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       }
     }
     __syncwarp();
-    // the weighted sums of the parts' O rows, then the stores; the merge slot
-    // is released last.  The parts present are block subsets 0 .. nw - 1 (a
-    // subset has blocks when c < nb).  This code runs once per piece, so it is
-    // kept compact: cold in the instruction cache, an unrolled form costs more
-    // in fetches than its loads.
-    const int nw = min(kWarps, inf->nb);
+    // the weighted sums of the parts' O rows, each written back over part
+    // 0's element (read by this lane only), then the stores from there; the
+    // merge slot is released last.  No global store is issued among the
+    // shared-memory loads of the sums, where it would hold them up.
+    const uint32_t part0 = sbase + LY::mo_off;
+    auto sums = [&](auto all_parts) {
+      constexpr bool kAll = decltype(all_parts)::value;
+      for (int e = lane; e < rows * D4; e += 32) {
+        const int i = e / D4, d4 = e % D4;
+        const uint32_t wrow = sbase + LY::mm_off + i * 4;
+        const uint32_t orow = part0 + (i * kOStride + 4 * d4) * 4;
+        // in batches of parts, every load of a batch issued before its sums
+        // (a part past nw reads stale bytes, replaced by 0)
+        constexpr int kB = kWarps > 6 ? (kWarps + 1) / 2 : kWarps;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int b = 0; b < kWarps; b += kB) {
+          float wt[kB];
+          float4 v[kB];
+#pragma unroll
+          for (int k = 0; k < kB && b + k < kWarps; ++k) {
+            wt[k] = __uint_as_float(lds32(wrow + (b + k) * (kMaxRows * 4)));
+            v[k] = lds_f4(orow + (b + k) * (kMaxRows * kOStride * 4));
+          }
+#pragma unroll
+          for (int k = 0; k < kB && b + k < kWarps; ++k) {
+            const bool has = kAll || b + k < nw;
+            acc.x = fmaf(has ? v[k].x : 0.f, wt[k], acc.x);
+            acc.y = fmaf(has ? v[k].y : 0.f, wt[k], acc.y);
+            acc.z = fmaf(has ? v[k].z : 0.f, wt[k], acc.z);
+            acc.w = fmaf(has ? v[k].w : 0.f, wt[k], acc.w);
+          }
+        }
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(orow), "f"(acc.x),
+                     "f"(acc.y), "f"(acc.z), "f"(acc.w)
+                     : "memory");
+      }
+    };
+    if (nw == kWarps) sums(std::true_type{});
+    else sums(std::false_type{});
     for (int e = lane; e < rows * D4; e += 32) {
       const int i = e / D4, d4 = e % D4;
-      const float* wrow = msl_m + i;
-      const float* orow = msl_o + i * kOStride + 4 * d4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      int w = rot;
-#pragma unroll 4
-      for (int c = 0; c < nw; ++c) {
-        const float wt = wrow[w * kMaxRows];
-        const float4 v = *reinterpret_cast<const float4*>(orow + w * (kMaxRows * kOStride));
-        acc.x = fmaf(v.x, wt, acc.x);
-        acc.y = fmaf(v.y, wt, acc.y);
-        acc.z = fmaf(v.z, wt, acc.z);
-        acc.w = fmaf(v.w, wt, acc.w);
-        w = w + 1 == kWarps ? 0 : w + 1;
-      }
+      const float4 acc = lds_f4(part0 + (i * kOStride + 4 * d4) * 4);
       const float Ls = row_l[i];
       if (direct) {
         const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
         const int gi = row0 + i;
-        const int64_t tok = q0 + gi / G, head = (int64_t)kvh * G + gi % G;
+        // one query token: its rows are consecutive heads of the kv-head
+        const int64_t tok = ql == 1 ? q0 : q0 + gi / G;
+        const int64_t head = (int64_t)kvh * G + (ql == 1 ? gi : gi % G);
         uint2 pk;
         pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
         pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
