@@ -118,9 +118,9 @@ struct DecodeLayout {
   static constexpr int mm_off = ring_off + ring_bytes;                // [kWarps][kMaxRows]
   static constexpr int ml_off = mm_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows]
   static constexpr int mo_off = ml_off + kWarps * kMaxRows * 4;       // [kWarps][kMaxRows][kOStride]
-  // the merged rows' max and sum
-  static constexpr int rs_off = mo_off + kWarps * kMaxRows * kOStride * 4;  // [2][kMaxRows]
-  static constexpr int merge_end = rs_off + 2 * kMaxRows * 4;
+  // the merged rows' max, sum and 1 / sum
+  static constexpr int rs_off = mo_off + kWarps * kMaxRows * kOStride * 4;  // [3][kMaxRows]
+  static constexpr int merge_end = rs_off + 3 * kMaxRows * 4;
   // two piece slots: info, block ids, query rows
   static constexpr int kInfoBytes = 64;
   static constexpr int kIdsBytes = kDecodeMaxPieceBlocks * 4;
@@ -257,6 +257,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   float* msl_o = reinterpret_cast<float*>(smem + LY::mo_off);
   float* row_m = reinterpret_cast<float*>(smem + LY::rs_off);
   float* row_l = row_m + kMaxRows;
+  float* row_inv = row_l + kMaxRows;
   int* meta = reinterpret_cast<int*>(smem + LY::meta_off);  // [kWarps][kStages][2]
   const uint32_t bars = sbase + LY::bar_off;                 // [kWarps][kStages] mbarriers
   volatile int* vabort = &ctl.abort;
@@ -667,6 +668,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       if (wg == 0) {
         row_m[i] = M;
         row_l[i] = Ls;
+        row_inv[i] = Ls > 0.f ? 1.f / Ls : 0.f;
       }
     }
     __syncwarp();
@@ -710,24 +712,33 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     };
     if (nw == kWarps) sums(std::true_type{});
     else sums(std::false_type{});
-    for (int e = lane; e < rows * D4; e += 32) {
-      const int i = e / D4, d4 = e % D4;
-      const float4 acc = lds_f4(part0 + (i * kOStride + 4 * d4) * 4);
-      const float Ls = row_l[i];
-      if (direct) {
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+    __syncwarp();
+    if (direct) {  // 8 dims (16 bytes of output) per lane and store
+      constexpr int D8 = D / 8;
+      for (int e = lane; e < rows * D8; e += 32) {
+        const int i = e / D8, d8 = e % D8;
+        const float4 a0 = lds_f4(part0 + (i * kOStride + 8 * d8) * 4);
+        const float4 a1 = lds_f4(part0 + (i * kOStride + 8 * d8 + 4) * 4);
+        const float inv = row_inv[i];
         const int gi = row0 + i;
         // one query token: its rows are consecutive heads of the kv-head
         const int64_t tok = ql == 1 ? q0 : q0 + gi / G;
         const int64_t head = (int64_t)kvh * G + (ql == 1 ? gi : gi % G);
-        uint2 pk;
-        pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-        pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-        *reinterpret_cast<uint2*>(out + (tok * p.num_q_heads + head) * D + 4 * d4) = pk;
-      } else {
-        reinterpret_cast<float4*>(p.ws_o)[(slot0 + i) * D4 + d4] = acc;
-        if (d4 == 0) reinterpret_cast<float2*>(p.ws_ml)[slot0 + i] = make_float2(row_m[i], Ls);
+        uint4 pk;
+        pk.x = pack_bf16x2(a0.x * inv, a0.y * inv);
+        pk.y = pack_bf16x2(a0.z * inv, a0.w * inv);
+        pk.z = pack_bf16x2(a1.x * inv, a1.y * inv);
+        pk.w = pack_bf16x2(a1.z * inv, a1.w * inv);
+        *reinterpret_cast<uint4*>(out + (tok * p.num_q_heads + head) * D + 8 * d8) = pk;
       }
+    } else {
+      for (int e = lane; e < rows * D4; e += 32) {
+        const int i = e / D4, d4 = e % D4;
+        reinterpret_cast<float4*>(p.ws_o)[(slot0 + i) * D4 + d4] =
+            lds_f4(part0 + (i * kOStride + 4 * d4) * 4);
+      }
+      if (lane < rows)
+        reinterpret_cast<float2*>(p.ws_ml)[slot0 + lane] = make_float2(row_m[lane], row_l[lane]);
     }
     __syncwarp();  // every lane is done with the merge slot and the piece slot
     if (lane == 0) {
