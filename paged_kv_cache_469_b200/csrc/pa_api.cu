@@ -165,11 +165,14 @@ extern "C" int pa_workspace_init(void* workspace, size_t workspace_bytes,
 
 namespace {
 
-// Rates one SM sustains on its own, used only to split the SMs between the
-// two classes of a mixed step: the tensor-core prefill kernel (bf16 flops of
-// unmasked query-key pairs per second) and the decode kernel (K/V bytes per
-// second when every SM streams).
-constexpr double kPrefillFlopsPerSm = 5.0e12;
+// Rates one SM sustains while the two classes of a mixed step share the GPU,
+// used only to split the SMs between them: the tensor-core prefill kernel
+// (bf16 flops of unmasked query-key pairs per second; 5.5e12 when it has the
+// GPU to itself, less beside a decode grid that keeps HBM busy) and the decode
+// kernel (K/V bytes per second when every SM streams).  Measured on the
+// Llama-3-8B mixed step: 3.3e12 to 4e12 (23 to 27 prefill SMs) gave the
+// shortest step, 5e12 9 % longer, 6e12 16 % longer.
+constexpr double kPrefillFlopsPerSm = 3.7e12;
 constexpr double kDecodeBytesPerSm = 46.0e9;
 
 // A side stream and two events, per thread and device, for the calls that run
