@@ -1,6 +1,7 @@
 // pa_tma.cuh -- tensor-memory-accelerator (TMA) loads shared by the kernels of
 // libpa.so: the device-side copy instruction and the host-side tensor maps of
-// the paged K/V pool.  No load here uses cluster multicast.
+// the paged K/V pool.  Every load here fills only the issuing CTA's own shared
+// memory.
 #pragma once
 
 #include <cuda.h>
