@@ -991,7 +991,7 @@ __host__ __device__ __forceinline__ int4 make_piece(int s, int kvh, int rg, int 
 // One CTA: the piece list of every decode-class sequence, written to the
 // workspace (count, blocks per piece, then the pieces, largest first).
 __global__ void __launch_bounds__(1024)
-decode_plan_kernel(const AttnParams p, int ctas, int head_dim) {
+decode_plan_kernel(const AttnParams p, int ctas, int head_dim, int whole_units) {
   __shared__ unsigned long long sh_total;
   __shared__ int sh_max_nblk, sh_P, sh_full, sh_count;
   __shared__ int hist[kDecodeMaxPieceBlocks + 1];  // tail pieces by size, then offsets
@@ -1022,8 +1022,9 @@ decode_plan_kernel(const AttnParams p, int ctas, int head_dim) {
   atomicMax(&sh_max_nblk, mx);
   __syncthreads();
   if (threadIdx.x == 0)
-    sh_P = choose_piece_blocks((long long)sh_total, sh_max_nblk, ctas,
-                               p.max_parts / max(1, p.row_groups), head_dim);
+    sh_P = whole_units ? max(1, sh_max_nblk)
+                       : choose_piece_blocks((long long)sh_total, sh_max_nblk, ctas,
+                                             p.max_parts / max(1, p.row_groups), head_dim);
   __syncthreads();
   const int P = sh_P;
   // pass 2: count the full pieces and the tail pieces by size
@@ -1137,6 +1138,9 @@ bool host_piece_list(DecodeWork* work, const AttnParams& p, const int32_t* seq_l
 // nearly done.  (The claims of a shared counter adapt to SMs that run slower,
 // but every claim's round trips and staging then sit on the CTA's path.)
 constexpr int kDecodeDealPiecesPerCta = 4;
+// a device-listed launch keeps units whole when no unit can exceed this many
+// blocks (by the host's bound on the lengths)
+constexpr int kDecodeWholeUnitBlocks = 256;
 
 void deal_pieces(DecodeWork* work, int ctas) {
   const int n = work->count, P = work->piece_blocks;
@@ -1280,10 +1284,19 @@ cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_
     // it, the claims' adapting to each SM's actual pace is worth more.
     if (ctas == full && work.count >= kDecodeDealPiecesPerCta * grid) deal_pieces(&work, grid);
   } else {
+    // Listed on the device.  When the host's bound on the lengths keeps every
+    // unit short and there are at least as many units as CTAs, the units stay
+    // whole (the claims balance them), so no partial needs merging and the
+    // combine kernel is not launched.
+    const long long bound_blocks =
+        (min((long long)p.max_seq_len, (long long)p.max_blocks_per_seq * kBlockSize) +
+         kBlockSize - 1) / kBlockSize;
+    const long long units = (long long)p.num_seqs * p.num_kv_heads * p.row_groups;
+    const int whole = bound_blocks <= kDecodeWholeUnitBlocks && units >= ctas;
     work.count = 0;
     work.piece_blocks = 0;
     work.from_ws = 1;
-    work.split = 1;
+    work.split = !whole;
     work.dealt = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
@@ -1294,7 +1307,7 @@ cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_plan_kernel, p, ctas, head_dim);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_plan_kernel, p, ctas, head_dim, whole);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e;
@@ -1306,7 +1319,7 @@ cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_
     e = wc ? launch_rows<128, true>(p, work, grid, max_rows, stream)
            : launch_rows<128, false>(p, work, grid, max_rows, stream);
   if (e != cudaSuccess) return e;
-  if (work.from_ws || work.split) {
+  if (work.split) {
     // the units cut into several pieces: merge their partials
     const long units = (long)p.num_seqs * p.num_kv_heads * p.row_groups;
     cudaLaunchConfig_t cfg = {};
