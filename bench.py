@@ -549,10 +549,11 @@ def bench_planner(args, dev, stream) -> dict:
 
 def bench_device_loop(args, dev, stream, world, clocks) -> dict:
     """The serving loop planned on the GPU: every step is pa_plan_step (one
-    token more per sequence), pa_attention_varlen_write_cache without host
-    copies (its decode work listed on the device) and the new lengths copied
-    into num_computed, for the decode workload's 64 sequences, starting from
-    its contexts.  --steps such steps are captured as one CUDA graph, rotating
+    token more per sequence) and pa_attention_varlen_write_cache without host
+    copies (its decode work listed on the device), for the decode workload's 64
+    sequences, starting from its contexts.  The lengths alternate between two
+    buffers: a step's new lengths are the next step's num_computed (the two
+    never alias, as pa_plan_step requires).  --steps such steps are captured as one CUDA graph, rotating
     over the same copies of the workload as the main leg, and timed as one
     replay.  Query tokens/s (one per sequence and step), and KV GB/s on the
     keys the steps actually read (the sequences grow by one token per step)."""
@@ -572,9 +573,9 @@ def bench_device_loop(args, dev, stream, world, clocks) -> dict:
         st = {"d": d,
               "fq": torch.from_numpy(step.free_queue).to(dev),
               "state": lib.new_planner_state(d.plan.blocks_taken, device=dev),
-              "num_computed": d.seq_lens.clone(),
+              "lens": [d.seq_lens.clone(), torch.empty(S, dtype=torch.int32, device=dev)],
+              "flip": 0,  # lens[flip] holds the lengths computed so far
               "query_lens": torch.ones(S, dtype=torch.int32, device=dev),
-              "seq_lens": torch.empty(S, dtype=torch.int32, device=dev),
               "qsl": torch.empty(S + 1, dtype=torch.int32, device=dev),
               "slots": torch.empty(S, dtype=torch.int64, device=dev),
               "ws": lib.new_workspace(S, step.num_q_heads, step.num_kv_heads, step.head_dim,
@@ -585,13 +586,16 @@ def bench_device_loop(args, dev, stream, world, clocks) -> dict:
         d = st["d"]
 
         def call():
-            lib.plan_step(st["fq"], st["state"], st["num_computed"], st["query_lens"],
-                          d.block_tables, st["seq_lens"], st["qsl"], st["slots"])
+            # (the buffers alternate call by call in the order the calls run:
+            # eagerly, or as recorded in a graph that is replayed once)
+            done, new = st["lens"][st["flip"]], st["lens"][1 - st["flip"]]
+            lib.plan_step(st["fq"], st["state"], done, st["query_lens"], d.block_tables, new,
+                          st["qsl"], st["slots"])
             lib.attention_varlen_write_cache(
                 d.out, d.q, d.k_new, d.v_new, d.k_cache, d.v_cache, st["slots"], d.block_tables,
-                st["seq_lens"], st["qsl"], max_query_len=1, max_seq_len=bound,
-                scale=step.scale, workspace=st["ws"])
-            st["num_computed"].copy_(st["seq_lens"])
+                new, st["qsl"], max_query_len=1, max_seq_len=bound, scale=step.scale,
+                workspace=st["ws"])
+            st["flip"] ^= 1
         return call
 
     calls = [call_for(st) for st in loops]
@@ -622,8 +626,8 @@ def bench_device_loop(args, dev, stream, world, clocks) -> dict:
             "value": round(tokens / (ms / 1e3), 1), "unit": "query tokens/s",
             "kv_gbs": round(sum_over_ranks(kv, world) / args.steps / (ms / 1e3) / 1e9, 1),
             "launch": ("one CUDA graph of --steps steps, each pa_plan_step + "
-                       "pa_attention_varlen_write_cache (no host copies) + a copy of the new "
-                       "lengths; no host work between steps")}
+                       "pa_attention_varlen_write_cache (no host copies), the lengths in two "
+                       "alternating buffers; no host work between steps")}
 
 
 def capture_e2e(dss, host_ins, host_out, k: int):
