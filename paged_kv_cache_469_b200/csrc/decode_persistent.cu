@@ -502,6 +502,34 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   int n_issued = 0, n_comp = 0;
   uint32_t bad = 0;  // bit (stage): that stage's block id was outside the pool
 
+  // The copies of block i of piece pc (id: its cache block, kvh: the piece's
+  // kv-head) into the next ring stage.
+  auto issue_stage = [&](int pc, int i, int id, int kvh) {
+    const int st = n_issued % kStages;
+    // a block id outside the pool is never dereferenced: the box is read from
+    // past the tensor's extent (zeros) and its keys are masked
+    const bool id_ok = id >= 0 && id < p.num_blocks;
+    if (id_ok) bad &= ~(1u << st);
+    else bad |= 1u << st;
+    const int row_bh = id_ok ? id * p.num_kv_heads + kvh : oob_bh;
+    if (lane == 0) {
+      const uint32_t ks = ring + st * LY::kStageBytes;
+      const uint32_t bar = bars + 8 * (warp * kStages + st);
+      // (the warp's earlier reads of this stage have completed: their values
+      // went into MMAs before the stage was freed)
+      mbar_expect_tx(bar, LY::kStageBytes);
+#pragma unroll
+      for (int pn = 0; pn < kPanels; ++pn) {
+        tma_load_3d(ks + pn * 2048, &tm_k, 64 * pn, 0, row_bh, bar);
+        tma_load_3d(ks + LY::kTileBytes + pn * 2048, &tm_v, 64 * pn, 0, row_bh, bar);
+      }
+    }
+    // (every lane stores the same values and reads back only what it stored)
+    my_meta[2 * st] = pc;
+    my_meta[2 * st + 1] = i;
+    ++n_issued;
+  };
+
   // Issue the copies of this warp's next block; false when there is none yet
   // (the next piece is not published and `block` is false) or none at all.
   // Warp w takes the blocks c, c + kWarps, ... of every piece, c = (w - rot)
@@ -536,30 +564,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       ++ip;
       ii = -1;
     }
-    const int st = n_issued % kStages;
-    const int id = slot_ids(ip)[ii];
-    // a block id outside the pool is never dereferenced: the box is read from
-    // past the tensor's extent (zeros) and its keys are masked
-    const bool id_ok = id >= 0 && id < p.num_blocks;
-    if (id_ok) bad &= ~(1u << st);
-    else bad |= 1u << st;
-    const int row_bh = id_ok ? id * p.num_kv_heads + inf->kvh : oob_bh;
-    if (lane == 0) {
-      const uint32_t ks = ring + st * LY::kStageBytes;
-      const uint32_t bar = bars + 8 * (warp * kStages + st);
-      // (the warp's earlier reads of this stage have completed: their values
-      // went into MMAs before the stage was freed)
-      mbar_expect_tx(bar, LY::kStageBytes);
-#pragma unroll
-      for (int pn = 0; pn < kPanels; ++pn) {
-        tma_load_3d(ks + pn * 2048, &tm_k, 64 * pn, 0, row_bh, bar);
-        tma_load_3d(ks + LY::kTileBytes + pn * 2048, &tm_v, 64 * pn, 0, row_bh, bar);
-      }
-    }
-    // (every lane stores the same values and reads back only what it stored)
-    my_meta[2 * st] = ip;
-    my_meta[2 * st + 1] = ii;
-    ++n_issued;
+    issue_stage(ip, ii, slot_ids(ip)[ii], inf->kvh);
     ii += kWarps;
     return true;
   };
@@ -749,6 +754,35 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     return true;
   };
 
+  // The CTA's first piece, when the list is in the kernel parameters: the
+  // warp's first blocks of it are issued straight from the block table (the
+  // piece's rotation is 0), while the scheduler stages the piece, so the
+  // first K/V tiles are on their way one round trip earlier.  Blocks that
+  // receive this step's new K/V rows are left to the normal path, which
+  // issues them only after the scheduler has written those rows.
+  if (!work.from_ws) {
+    const int gb = work.dealt ? work.cta_off[blockIdx.x] : (int)blockIdx.x;
+    const int ge = work.dealt ? work.cta_off[blockIdx.x + 1] : work.count;
+    if (gb < ge) {
+      const int4 it = work.items[gb];
+      const int s0 = it.x, j0 = it.y & 0xfff, kvh0 = (it.y >> 12) & 0x3ff;
+      const int ql0 = (it.y >> 24) & 0x7f, L0 = it.z;
+      const int P0 = work.piece_blocks;
+      const int blk_begin = j0 * P0;
+      const int nb0 = min(P0, (L0 + kBlockSize - 1) / kBlockSize - blk_begin);
+      const int lim = kWriteCache ? min(nb0, max(0, (L0 - ql0) / kBlockSize - blk_begin)) : nb0;
+      const int32_t* table = p.block_tables + (int64_t)s0 * p.max_blocks_per_seq + blk_begin;
+      int id = 0;
+      if (lane < kStages && warp + lane * kWarps < lim) id = table[warp + lane * kWarps];
+#pragma unroll
+      for (int k = 0; k < kStages; ++k) {
+        const int idk = __shfl_sync(0xffffffffu, id, k);
+        if (warp + k * kWarps < lim) issue_stage(0, warp + k * kWarps, idk, kvh0);
+      }
+      ii = warp + n_issued * kWarps;  // the next block of the piece to issue
+    }
+  }
+
   while (true) {
     // keep kStages blocks in flight; wait for a piece to be published only
     // when nothing is in flight
@@ -762,6 +796,9 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
 
     const int st = n_comp % kStages;
     const int pc = my_meta[2 * st], i = my_meta[2 * st + 1];
+    // (a block issued before its piece was published: the piece's query rows
+    // and fields are read once it is)
+    if (pc > seen && !spin_until([&] { return slot_state(pc) == 1; }, vabort, status)) break;
     const PieceInfo* inf = slot_info(pc);
     const int L = inf->L;
     if (pc != cur) {
