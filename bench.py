@@ -49,8 +49,8 @@ REFERENCE_BUDGET_S = 120.0  # host seconds the --impl reference steps may take i
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of DECODE_KERNEL
 # on this workload, from an ncu capture of that launch; None whenever that
 # kernel has changed since it was last captured
-DECODE_TRAFFIC_BYTES = 70_402_304  # ncu --set full, third launch of run_workload decode_tinyllama
-DECODE_KERNEL = "decode_persistent_kernel<64,8,false>"
+DECODE_TRAFFIC_BYTES = 70_217_472  # ncu --set full, third launch of run_workload decode_tinyllama
+DECODE_KERNEL = "decode_persistent_kernel<64,8,false,false>"
 KERNELS_PER_DECODE_STEP = 1  # the decode step is one launch (cache write inside the kernel)
 
 

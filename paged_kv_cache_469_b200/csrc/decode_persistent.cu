@@ -102,6 +102,8 @@ struct PieceInfo {
   int L, ql, q0;
   int rows, row0;  // this unit's query rows: global rows row0 .. row0 + rows - 1
   int rot;         // block subset c of the piece (blocks c, c + kWarps, ...) goes to warp (c + rot) % kWarps
+  int cw_tag;      // = tag once the step's new K/V rows of the piece are in the cache (write path)
+  int cw_first;    // the piece's first block receiving new rows (nb: none)
 };
 
 template <int D, int kMaxRows>
@@ -122,7 +124,7 @@ struct DecodeLayout {
   static constexpr int rs_off = mo_off + kWarps * kMaxRows * kOStride * 4;  // [3][kMaxRows]
   static constexpr int merge_end = rs_off + 3 * kMaxRows * 4;
   // two piece slots: info, block ids, query rows
-  static constexpr int kInfoBytes = 64;
+  static constexpr int kInfoBytes = 128;
   static constexpr int kIdsBytes = kDecodeMaxPieceBlocks * 4;
   static constexpr int kQBytes = kMaxRows * D * 2;
   static constexpr int kSlotBytes = kInfoBytes + kIdsBytes + kQBytes;
@@ -220,7 +222,14 @@ __device__ __forceinline__ int4 load_piece(const AttnParams& p, const DecodeWork
   return work.from_ws ? p.ws_pieces[g] : work.items[g];
 }
 
-template <int D, int kMaxRows, bool kWriteCache>
+// kWriteCache: the call writes the step's new K/V rows (the scheduler stores
+// them before the blocks holding them are read).  kLateRows (with it): a piece
+// is published before its rows are written, and the compute warps load the
+// blocks holding them only once the scheduler releases cw_tag; used when the
+// pieces are claimed, while pieces dealt on the host, staged well ahead of
+// their use, are written first and published after (that wait, compiled into
+// the issue path, measured 3 % slower on the prefix-cached step).
+template <int D, int kMaxRows, bool kWriteCache, bool kLateRows>
 __global__ void __launch_bounds__((DecodeCfg<D, kMaxRows>::kWarps + 1) * 32, 1)
 decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork work,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -270,6 +279,8 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
     ctl.passed[0] = ctl.passed[1] = 0;
     slot_info(0)->tag = -1;
     slot_info(1)->tag = -1;
+    slot_info(0)->cw_tag = -1;
+    slot_info(1)->cw_tag = -1;
     for (int i = 0; i < kWarps * kStages; ++i) mbar_init(bars + 8 * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tm_k);
@@ -362,6 +373,34 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       const int32_t* table = p.block_tables + (int64_t)s * p.max_blocks_per_seq + blk_begin;
       int* ids = slot_ids(pc);
       constexpr int kQv = (kMaxRows * kChunks + 31) / 32;  // 16-byte query loads per lane
+      // This step's new tokens of the sequence that fall in the piece's key
+      // range (the one-call path writes them into their cache slots, as
+      // pa_reshape_and_cache would): 16-byte chunks, K then V.  Lane t's
+      // first chunk is loaded with the block ids and the query rows (with
+      // kLateRows; otherwise when the rows are written).
+      int lo = 0, hi = 0;
+      if constexpr (kWriteCache) {
+        lo = max(L - ql, blk_begin * kBlockSize);
+        hi = min(L, (blk_begin + nb) * kBlockSize);
+      }
+      const int ncw = hi > lo ? (hi - lo) * kChunks : 0;  // chunks per K (and per V)
+      auto cw_src = [&](int i, bool& is_v, int& tok, int& c) {  // chunk i of the K and V rows
+        is_v = i >= ncw;
+        const int ii = is_v ? i - ncw : i;
+        tok = q0 + (lo - (L - ql)) + ii / kChunks;
+        c = ii % kChunks;
+        return ((int64_t)tok * p.num_kv_heads + kvh) * kChunks + c;
+      };
+      int64_t cw_slot = -1;
+      uint4 cw_val = make_uint4(0, 0, 0, 0);
+      bool cw_isv = false;
+      int cw_c = 0;
+      if (kLateRows && lane < 2 * ncw) {
+        int tok;
+        const int64_t src = cw_src(lane, cw_isv, tok, cw_c);
+        cw_slot = p.slot_mapping[tok];
+        cw_val = cw_isv ? ((const uint4*)p.v_new)[src] : ((const uint4*)p.k_new)[src];
+      }
       {
         const uint4* qg = (const uint4*)p.q;
         uint4 qv[kQv];
@@ -401,43 +440,6 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
             if (base + lane + 32 * k < nb) ids[base + lane + 32 * k] = iv[k];
         }
       }
-      if constexpr (kWriteCache) {
-        // This step's new tokens of the sequence that fall in the piece's key
-        // range go into their cache slots first (as pa_reshape_and_cache
-        // would); the compute warps read them only after the publication
-        // below.  With several 16-row groups, every row group's piece of the
-        // same (sequence, kv-head, blocks) stores the same bytes to the same
-        // slots, possibly while another CTA reads them: identical concurrent
-        // stores, so every read sees the new row.  No other piece reads
-        // these slots.
-        const int lo = max(L - ql, blk_begin * kBlockSize);
-        const int hi = min(L, (blk_begin + nb) * kBlockSize);
-        if (hi > lo) {
-          const int n = (hi - lo) * kChunks;
-          const int64_t num_slots = (int64_t)p.num_blocks * kBlockSize;
-          const uint4* kn = (const uint4*)p.k_new;
-          const uint4* vn = (const uint4*)p.v_new;
-          uint4* kcw = (uint4*)const_cast<void*>(p.k_cache);
-          uint4* vcw = (uint4*)const_cast<void*>(p.v_cache);
-          for (int i = lane; i < 2 * n; i += 32) {
-            const bool is_v = i >= n;
-            const int ii = is_v ? i - n : i;
-            const int r = ii / kChunks, c = ii % kChunks;
-            const int tok = q0 + (lo - (L - ql)) + r;
-            const int64_t slot = p.slot_mapping[tok];
-            if (slot < 0 || slot >= num_slots) continue;  // padding / out-of-pool slot
-            const int64_t dst =
-                ((slot / kBlockSize * p.num_kv_heads + kvh) * kBlockSize + slot % kBlockSize) *
-                    kChunks + c;
-            const int64_t src = ((int64_t)tok * p.num_kv_heads + kvh) * kChunks + c;
-            if (is_v) vcw[dst] = vn[src];
-            else kcw[dst] = kn[src];
-          }
-          // the compute warps read these rows with TMA (the async proxy)
-          __threadfence();
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-        }
-      }
       prev_nb = nb;
       if (lane == 0) {
         ctl.passed[pc & 1] = 0;
@@ -447,10 +449,47 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
         inf->L = L; inf->ql = ql; inf->q0 = q0;
         inf->rows = rows; inf->row0 = row0;
         inf->rot = rot;
+        inf->cw_first = ncw > 0 ? max(0, (L - ql) / kBlockSize - blk_begin) : nb;
       }
       rot = (rot + nb) % kWarps;
       __syncwarp();
+      auto write_rows = [&]() {
+        // With several 16-row groups, every row group's piece of the same
+        // (sequence, kv-head, blocks) stores the same bytes to the same slots,
+        // possibly while another CTA reads them: identical concurrent stores,
+        // so every read sees the new row.  No other piece reads these slots.
+        const int64_t num_slots = (int64_t)p.num_blocks * kBlockSize;
+        uint4* kcw = (uint4*)const_cast<void*>(p.k_cache);
+        uint4* vcw = (uint4*)const_cast<void*>(p.v_cache);
+        auto store = [&](int64_t slot, bool is_v, int c, const uint4& v) {
+          if (slot < 0 || slot >= num_slots) return;  // padding / out-of-pool slot
+          const int64_t dst =
+              ((slot / kBlockSize * p.num_kv_heads + kvh) * kBlockSize + slot % kBlockSize) *
+                  kChunks + c;
+          if (is_v) vcw[dst] = v;
+          else kcw[dst] = v;
+        };
+        if (kLateRows && lane < 2 * ncw) store(cw_slot, cw_isv, cw_c, cw_val);
+        for (int i = kLateRows ? lane + 32 : lane; i < 2 * ncw; i += 32) {  // (the rest)
+          bool is_v;
+          int tok, c;
+          const int64_t src = cw_src(i, is_v, tok, c);
+          const uint4 v = is_v ? ((const uint4*)p.v_new)[src] : ((const uint4*)p.k_new)[src];
+          store(p.slot_mapping[tok], is_v, c, v);
+        }
+        // the compute warps read these rows with TMA (the async proxy)
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) st_release(&inf->cw_tag, pc);
+      };
+      // With kLateRows the piece is published before the cache write (a
+      // release after the write would wait for its global stores), and only
+      // the blocks that receive new rows wait for cw_tag: the write's round
+      // trips then stay off the path of the piece's other blocks.
+      if (kWriteCache && !kLateRows && ncw > 0) write_rows();
       if (lane == 0) st_release(&inf->tag, pc);
+      if (kLateRows && ncw > 0) write_rows();
     }
     // the last CTA to finish claiming resets the claim counter for the next call
     if (lane == 0 && !dealt) {
@@ -498,6 +537,9 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   };
 
   int ip = 0, ii = -1;  // issue cursor: next candidate (piece, block of the piece; -1: its first)
+  // blocks receiving the step's new rows wait for them (kLateRows: the piece
+  // is published before the write)
+  constexpr bool cw_wait = kLateRows;
   bool issue_done = false;
   int n_issued = 0, n_comp = 0;
   uint32_t bad = 0;  // bit (stage): that stage's block id was outside the pool
@@ -563,6 +605,15 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       if (lane == 0 && first < inf->nb) atomicAdd(&ctl.passed[ip & 1], 1);
       ++ip;
       ii = -1;
+    }
+    // a block that receives the step's new rows is loaded only once the
+    // scheduler has written them (the piece is published before that write)
+    if (cw_wait && ii >= inf->cw_first && ld_acquire(&inf->cw_tag) < ip) {
+      if (!block) return false;
+      if (!spin_until([&] { return ld_acquire(&inf->cw_tag) >= ip; }, vabort, status)) {
+        issue_done = true;
+        return false;
+      }
     }
     issue_stage(ip, ii, slot_ids(ip)[ii], inf->kvh);
     ii += kWarps;
@@ -952,7 +1003,7 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
   }
 }
 
-template <int D, int kMaxRows, bool kWriteCache>
+template <int D, int kMaxRows, bool kWriteCache, bool kLateRows>
 cudaError_t launch_one(const AttnParams& p, const DecodeWork& work, int grid,
                        cudaStream_t stream) {
   using LY = DecodeLayout<D, kMaxRows>;
@@ -962,7 +1013,7 @@ cudaError_t launch_one(const AttnParams& p, const DecodeWork& work, int grid,
       !make_map(&tv, p.v_cache, D, kBlockSize, (uint64_t)p.num_blocks * p.num_kv_heads,
                 (uint64_t)D * 2, (uint64_t)kBlockSize * D * 2, kBlockSize, 1))
     return cudaErrorInvalidValue;
-  auto kernel = decode_persistent_kernel<D, kMaxRows, kWriteCache>;
+  auto kernel = decode_persistent_kernel<D, kMaxRows, kWriteCache, kLateRows>;
   static std::atomic<int> smem_done[64];
   cudaError_t e = raise_smem_limit(kernel, LY::total, smem_done);
   if (e != cudaSuccess) return e;
@@ -979,12 +1030,12 @@ cudaError_t launch_one(const AttnParams& p, const DecodeWork& work, int grid,
   return cudaLaunchKernelEx(&cfg, kernel, p, work, tk, tv);
 }
 
-template <int D, bool kWriteCache>
+template <int D, bool kWriteCache, bool kLateRows>
 cudaError_t launch_rows(const AttnParams& p, const DecodeWork& work, int grid, int max_rows,
                         cudaStream_t stream) {
-  if (max_rows <= 4) return launch_one<D, 4, kWriteCache>(p, work, grid, stream);
-  if (max_rows <= 8) return launch_one<D, 8, kWriteCache>(p, work, grid, stream);
-  return launch_one<D, 16, kWriteCache>(p, work, grid, stream);
+  if (max_rows <= 4) return launch_one<D, 4, kWriteCache, kLateRows>(p, work, grid, stream);
+  if (max_rows <= 8) return launch_one<D, 8, kWriteCache, kLateRows>(p, work, grid, stream);
+  return launch_one<D, 16, kWriteCache, kLateRows>(p, work, grid, stream);
 }
 
 // ------------------------------------------------------------------ piece lists
@@ -1279,7 +1330,7 @@ int max_ctas_one() {
   int n = cached[dev].load(std::memory_order_relaxed);
   if (n > 0) return n;
   using LY = DecodeLayout<D, kMaxRows>;
-  auto kernel = decode_persistent_kernel<D, kMaxRows, false>;
+  auto kernel = decode_persistent_kernel<D, kMaxRows, false, false>;
   static std::atomic<int> smem_done[64];
   int per_sm = 0;
   if (raise_smem_limit(kernel, LY::total, smem_done) != cudaSuccess ||
@@ -1349,12 +1400,15 @@ cudaError_t launch_decode(const AttnParams& p, int head_dim, const int32_t* seq_
   }
   cudaError_t e;
   const bool wc = p.slot_mapping != nullptr;
+  const bool late = !work.dealt;  // (the write path's pieces are claimed: kLateRows)
   if (head_dim == 64)
-    e = wc ? launch_rows<64, true>(p, work, grid, max_rows, stream)
-           : launch_rows<64, false>(p, work, grid, max_rows, stream);
+    e = !wc   ? launch_rows<64, false, false>(p, work, grid, max_rows, stream)
+        : late ? launch_rows<64, true, true>(p, work, grid, max_rows, stream)
+               : launch_rows<64, true, false>(p, work, grid, max_rows, stream);
   else
-    e = wc ? launch_rows<128, true>(p, work, grid, max_rows, stream)
-           : launch_rows<128, false>(p, work, grid, max_rows, stream);
+    e = !wc   ? launch_rows<128, false, false>(p, work, grid, max_rows, stream)
+        : late ? launch_rows<128, true, true>(p, work, grid, max_rows, stream)
+               : launch_rows<128, true, false>(p, work, grid, max_rows, stream);
   if (e != cudaSuccess) return e;
   if (work.split) {
     // the units cut into several pieces: merge their partials
