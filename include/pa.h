@@ -32,9 +32,9 @@
  *     PA_ERR_CUDA reports a failed launch (cudaGetLastError).
  *   - Calls can be captured in a CUDA graph.  A capture records the launch
  *     plan of that call: with the optional host copies of seq_lens and
- *     query_start_loc, that plan follows them (kernel choice, split-K
- *     partition length, the prefill work list), so a replay needs device
- *     arrays that still hold those values.
+ *     query_start_loc, that plan follows them (kernel choice, the decode
+ *     pieces, their order and their dealing to the CTAs, the prefill work
+ *     list), so a replay needs device arrays that still hold those values.
  *   - Nothing traps on the device.  Slots or block ids outside the pool are
  *     never dereferenced (see each call).
  *   - dtype is the element type of q, k, v, the caches and out alike.
@@ -159,9 +159,11 @@ int pa_workspace_init(void* workspace, size_t workspace_bytes, struct CUstream_s
  *   seq_lens_host, query_start_loc_host  optional (NULL) host copies of the
  *                  two device arrays, equal to them: when given, the call
  *                  checks them, launches only the kernels the step needs,
- *                  sizes the split-K partitions from the step's total keys,
- *                  and (up to 1024 prefill work items) passes the prefill work
- *                  list with the launch instead of building it on the GPU
+ *                  cuts the decode work into pieces sized from the step's
+ *                  total keys and passes their list (up to 1792 pieces) with
+ *                  the launch, and (up to 1024 prefill work items) passes the
+ *                  prefill work list with it, instead of building them on
+ *                  the GPU
  *
  * Decode-class sequences (q_len * num_q_heads / num_kv_heads <= 64 query
  * rows per kv-head: single-token decodes and the few-token queries of
