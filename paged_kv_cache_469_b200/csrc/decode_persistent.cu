@@ -19,24 +19,39 @@
 // CTAs); otherwise the long units are cut so that every CTA gets a few pieces.
 //
 // Grid.  One CTA per SM (its shared memory holds the streaming rings), each
-// running until the list is exhausted.  CTA b starts with piece b and claims
-// the next piece from a global counter once all blocks of its current piece
-// have been issued (their copies are still in flight while the claim and the
-// piece's staging complete), so the SMs that get through their work first
-// take the next pieces.  Inside a CTA:
+// running until its work is done.  Pieces reach the CTAs in one of two ways:
+//   claims  CTA b starts with piece b and claims the next piece from a global
+//       counter once every compute warp with blocks in its current piece has
+//       issued them all (their copies are still in flight while the claim
+//       and the piece's staging complete), so the SMs that get through their
+//       work first take the next pieces;
+//   dealt   when every SM has a CTA and the list holds at least a few pieces
+//       per CTA, the host deals the pieces to the CTAs beforehand (longest
+//       first, each to the CTA with the least work so far, a piece counting
+//       its blocks plus a fixed cost) and CTA b runs its own run of the list
+//       in order.
+// Inside a CTA:
 //
-//   scheduler warp (the last warp)  claims a piece, copies its block ids and
+//   scheduler warp (the last warp)  takes a piece, copies its block ids and
 //       its query rows into a shared-memory piece slot (two slots: piece p
-//       lives in slot p % 2), writes the step's new K/V rows of the piece into
-//       the cache first when the call asks for it, and publishes the slot.
-//   compute warps 0 .. kWarps-1     warp w takes blocks w, w + kWarps, ... of
-//       every piece.  It streams them through a private ring of kStages
-//       shared-memory stages (K tile + V tile of one (block, kv-head)) filled
-//       by TMA (16 x 64 boxes, one mbarrier per stage), up to kStages blocks
-//       in flight, and
-//       the ring runs on from one piece into the next without draining.  Per
-//       16-token block, with the keys on the MMA's M side and the (at most
-//       8 per n-tile) query rows on its N side, so that no MMA row is padding:
+//       lives in slot p % 2) and publishes the slot.  When the call also
+//       writes the step's new K/V rows, the scheduler stores the rows of a
+//       claimed piece after publishing it and then raises a second flag of
+//       the slot; a compute warp waits for that flag only before loading a
+//       block that receives new rows.  (For dealt pieces the rows are
+//       written before the slot is published.)
+//   compute warps 0 .. kWarps-1     block subset c of a piece (its blocks c,
+//       c + kWarps, ...) goes to warp (c + rot) % kWarps, where rot carries
+//       on from the previous piece so that no warp gets every piece's ragged
+//       remainder.  For the CTA's first piece the warps read their block ids
+//       from the block table themselves and issue their first loads (blocks
+//       receiving new rows excepted) before the slot is published.  Each warp streams its blocks through a
+//       private ring of kStages shared-memory stages (K tile + V tile of one
+//       (block, kv-head)) filled by TMA (16 x 64 boxes, one mbarrier per
+//       stage), up to kStages blocks in flight, and the ring runs on from one
+//       piece into the next without draining.  Per 16-token block, with the
+//       keys on the MMA's M side and the (at most 8 per n-tile) query rows on
+//       its N side, so that no MMA row is padding:
 //         S^T[16 keys x 8 rows]  = K . Q^T   mma.m16n8k16 per 16 dims of D
 //                                            (K by ldmatrix from the ring)
 //         online softmax down the columns of S^T (fp32 running max and sum,
@@ -45,8 +60,10 @@
 //         O^T[D x 8 rows]       += V^T . P^T  mma.m16n8k16 per 16 dims of D
 //                                            (V^T by ldmatrix.trans)
 //   piece merge  when a warp has computed its last block of a piece it puts
-//       its (max, sum, O) in a shared merge slot; the last warp to arrive
-//       merges them and stores the piece's result: the output rows when the
+//       its (max, sum, O) in a shared merge slot, at the place of its block
+//       subset; the warp whose blocks complete the piece's count merges the
+//       parts in subset order (so the result does not depend on timing) and
+//       stores the piece's result: the output rows when the
 //       piece is the whole unit, else an fp32 partial in the workspace.  No
 //       CTA ever waits for another, and no merge waits for global memory.
 //   combine kernel  (launched right after, as a programmatic dependent) one
@@ -57,8 +74,9 @@
 // shared memory (the TMA 128-byte swizzle) so that every 8 x 8 matrix that
 // ldmatrix reads hits eight distinct bank groups.
 //
-// Every wait on another warp of the CTA (a piece slot not yet published, the
-// merge slot still in use) is bounded by a time limit; one that runs out sets
+// Every wait on another warp of the CTA (a piece slot not yet published, a
+// block's new rows not yet written, the merge slot still in use, the warps
+// not yet past the current piece) is bounded by a time limit; one that runs out sets
 // the workspace status bit and the CTA winds down instead of hanging.  The
 // kernel is launched as a programmatic dependent of whatever precedes it on
 // the stream; before griddepcontrol.wait it reads only its own parameters.
