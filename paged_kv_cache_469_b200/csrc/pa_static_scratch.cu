@@ -98,8 +98,9 @@ extern "C" int pa_attention_varlen_static_scratch(
   if (rc != PA_OK) return rc;
   if (num_seqs > 0 && num_tokens > 0) {
     // The array still holds whatever the previous call left there, possibly
-    // under another layout: the status word and the split-K arrival counters
-    // must start at zero, so clear them (everything before the partials).
+    // under another layout: the status word and the decode grid's claim
+    // counters must start at zero, so clear them (everything before the
+    // partials).
     const pa::WorkspaceLayout w =
         pa::workspace_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_seq_len);
     if (cudaMemsetAsync(scratch, 0, w.o_off, (cudaStream_t)stream) != cudaSuccess)
