@@ -395,7 +395,11 @@ decode_persistent_kernel(const AttnParams p, const __grid_constant__ DecodeWork 
       // range (the one-call path writes them into their cache slots, as
       // pa_reshape_and_cache would): 16-byte chunks, K then V.  Lane t's
       // first chunk is loaded with the block ids and the query rows (with
-      // kLateRows; otherwise when the rows are written).
+      // kLateRows; otherwise when the rows are written).  When a unit's
+      // query rows span several row groups, the pieces of each row group
+      // over these keys store the same rows: identical bytes, so a CTA that
+      // has completed its own stores reads the new values whatever the
+      // others' stores are doing.
       int lo = 0, hi = 0;
       if constexpr (kWriteCache) {
         lo = max(L - ql, blk_begin * kBlockSize);
